@@ -1,0 +1,192 @@
+"""Seeded synthetic inputs for MLA latent-cache decode.
+
+This module only draws random numbers and lays them out in memory (a paged
+latent pool plus a block table). It holds none of the attention arithmetic, so
+both the CPU oracle (via the tests) and the CUDA path can consume the same
+inputs without sharing any of the method's code.
+
+Workloads (shapes as the TransMLA / TPLA pages describe the models; values are
+synthetic because no trained weights are available):
+
+* ``tiny``        fp32, 8 heads, r=64, rope 16, nope 32, v 32, L=256, contiguous
+* ``llama2_7b``   bf16, TransMLA-converted LLaMA-2-7B shape: 32 heads, r=512,
+                  rope 64, nope 128, v 128 (576 cached values per token against
+                  8192 for the GQA original), B=16, L=8192, paged
+* ``deepseek_v3`` bf16, 128 heads, r=512, rope 64, nope 128, v 128, B=32,
+                  L=32768, paged
+* ``kimi_k2_mtp`` bf16, 64 heads, same dims, 64 sequences with L uniform in
+                  [1024, 32768], 2 causal query tokens per sequence, paged
+* ``tpla_dsv3``   bf16, DeepSeek-V3 shape with the latent split into 2 shards
+                  (TPLA), B=32, L=32768, paged
+
+Recipe (every draw is float32 N(0, 1) from ``torch.Generator`` seeded per
+tensor, then scaled and cast to the workload dtype with round-to-nearest-even):
+
+* per-tensor seeds: ``seed * 1_000_003 + tag`` with a fixed tag per tensor;
+  the latent rows of sequence ``b`` use tag ``100 + b`` so that any subset of
+  sequences can be regenerated on its own;
+* lengths (varlen only): integers uniform in [lo, hi] inclusive;
+* q_nope [B, Lq, H, dn], q_rope [B, Lq, H, dr] ~ N(0, 1) (q_rope stands for the
+  query after RoPE; decode applies no rotation);
+* per sequence, one [L_b, r + dr] block ~ N(0, 1): columns [0, r) are cKV,
+  columns [r, r + dr) are the (already rotated) decoupled RoPE key;
+* W_UK [H, dn, r] and W_UV [H, r, dv] ~ N(0, 1/r) with r the full latent rank;
+* the pool has sum_b ceil(L_b / P) blocks of P = 64 tokens; paged workloads
+  place logical page (b, i) at a block chosen by a seeded random permutation,
+  contiguous ones at the identity position. Unused table entries are -1 and
+  the tail of a partial page is zero.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = ["Workload", "WORKLOADS", "generate", "logical_cache", "pages_of"]
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    seed: int
+    batch: int
+    q_len: int
+    heads: int
+    latent_rank: int
+    rope_dim: int
+    nope_dim: int
+    v_dim: int
+    context: int            # fixed length, or the upper bound when varlen
+    context_min: int = 0    # > 0 selects uniform integer lengths in [context_min, context]
+    latent_shards: int = 1
+    dtype: str = "bf16"     # "bf16" or "fp32"
+    paged: bool = True      # False: identity block table (contiguous cache)
+    page_size: int = 64
+
+    @property
+    def softmax_scale(self) -> float:
+        # 1/sqrt(d_qk) with d_qk = nope + rope dims of the non-absorbed head
+        return 1.0 / math.sqrt(self.nope_dim + self.rope_dim)
+
+    @property
+    def row_width(self) -> int:
+        return self.latent_rank + self.rope_dim
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", seed=0, batch=1, q_len=1, heads=8, latent_rank=64,
+                     rope_dim=16, nope_dim=32, v_dim=32, context=256,
+                     dtype="fp32", paged=False),
+    "llama2_7b": Workload("llama2_7b", seed=1, batch=16, q_len=1, heads=32,
+                          latent_rank=512, rope_dim=64, nope_dim=128, v_dim=128,
+                          context=8192),
+    "deepseek_v3": Workload("deepseek_v3", seed=2, batch=32, q_len=1, heads=128,
+                            latent_rank=512, rope_dim=64, nope_dim=128, v_dim=128,
+                            context=32768),
+    "kimi_k2_mtp": Workload("kimi_k2_mtp", seed=3, batch=64, q_len=2, heads=64,
+                            latent_rank=512, rope_dim=64, nope_dim=128, v_dim=128,
+                            context=32768, context_min=1024),
+    "tpla_dsv3": Workload("tpla_dsv3", seed=4, batch=32, q_len=1, heads=128,
+                          latent_rank=512, rope_dim=64, nope_dim=128, v_dim=128,
+                          context=32768, latent_shards=2),
+}
+
+_TAG_LENS, _TAG_QN, _TAG_QR, _TAG_WUK, _TAG_WUV, _TAG_PERM = 1, 2, 3, 4, 5, 6
+_TAG_SEQ0 = 100
+
+
+def _gen(seed: int, tag: int) -> torch.Generator:
+    g = torch.Generator()
+    g.manual_seed(seed * 1_000_003 + tag)
+    return g
+
+
+def pages_of(length: int, page_size: int) -> int:
+    return (length + page_size - 1) // page_size
+
+
+def draw_lengths(wl: Workload) -> torch.Tensor:
+    if wl.context_min > 0:
+        g = _gen(wl.seed, _TAG_LENS)
+        return torch.randint(wl.context_min, wl.context + 1, (wl.batch,),
+                             generator=g, dtype=torch.int64).to(torch.int32)
+    return torch.full((wl.batch,), wl.context, dtype=torch.int32)
+
+
+def draw_sequence_rows(wl: Workload, b: int, length: int) -> torch.Tensor:
+    """[length, r + dr] latent rows of sequence b in the workload dtype."""
+    g = _gen(wl.seed, _TAG_SEQ0 + b)
+    x = torch.randn((length, wl.row_width), generator=g, dtype=torch.float32)
+    return x.to(wl.torch_dtype)
+
+
+def generate(wl: Workload, seq_lens: Optional[Sequence[int]] = None,
+             with_pool: bool = True) -> dict:
+    """All decode inputs as CPU tensors.
+
+    ``seq_lens`` overrides the workload's lengths (reduced-size parity cases).
+    Returns q_nope, q_rope, w_uk, w_uv, seq_lens (int32), and when
+    ``with_pool``: kv_pool [num_blocks, P, r + dr], block_table [B, max_pages]
+    (int32, -1 where unused), num_blocks.
+    """
+    if seq_lens is None:
+        lens = draw_lengths(wl)
+    else:
+        lens = torch.as_tensor(list(seq_lens), dtype=torch.int32)
+    B = int(lens.numel())
+    dt = wl.torch_dtype
+    r, dr, dn, dv, H, Lq = (wl.latent_rank, wl.rope_dim, wl.nope_dim, wl.v_dim,
+                            wl.heads, wl.q_len)
+    out = {"seq_lens": lens}
+    out["q_nope"] = torch.randn((B, Lq, H, dn), generator=_gen(wl.seed, _TAG_QN)).to(dt)
+    out["q_rope"] = torch.randn((B, Lq, H, dr), generator=_gen(wl.seed, _TAG_QR)).to(dt)
+    wstd = 1.0 / math.sqrt(r)
+    out["w_uk"] = (torch.randn((H, dn, r), generator=_gen(wl.seed, _TAG_WUK)) * wstd).to(dt)
+    out["w_uv"] = (torch.randn((H, r, dv), generator=_gen(wl.seed, _TAG_WUV)) * wstd).to(dt)
+    if not with_pool:
+        return out
+
+    P = wl.page_size
+    npages = [pages_of(int(L), P) for L in lens.tolist()]
+    total = sum(npages)
+    max_pages = max(npages) if npages else 0
+    if wl.paged:
+        perm = torch.randperm(total, generator=_gen(wl.seed, _TAG_PERM)).to(torch.int32)
+    else:
+        perm = torch.arange(total, dtype=torch.int32)
+    table = torch.full((B, max(max_pages, 1)), -1, dtype=torch.int32)
+    pool = torch.zeros((total, P, wl.row_width), dtype=dt)
+    base = 0
+    for b, L in enumerate(lens.tolist()):
+        n = npages[b]
+        ids = perm[base:base + n]
+        table[b, :n] = ids
+        rows = draw_sequence_rows(wl, b, L)
+        padded = torch.zeros((n * P, wl.row_width), dtype=dt)
+        padded[:L] = rows
+        pool[ids.long()] = padded.view(n, P, wl.row_width)
+        base += n
+    out["kv_pool"] = pool
+    out["block_table"] = table
+    out["num_blocks"] = total
+    return out
+
+
+def logical_cache(inputs: dict, b: int, wl: Workload):
+    """(cKV [L_b, r], k_rope [L_b, dr]) of sequence b, gathered from the pool."""
+    L = int(inputs["seq_lens"][b])
+    P = wl.page_size
+    n = pages_of(L, P)
+    ids = inputs["block_table"][b, :n].long()
+    rows = inputs["kv_pool"][ids].reshape(n * P, wl.row_width)[:L]
+    return rows[:, :wl.latent_rank], rows[:, wl.latent_rank:]
