@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Benchmark of one MLA decode step over a paged latent KV cache on B200.
+
+A step is one call of the C ABI's mla_decode_run on one batch: the absorb
+kernel, the split-KV latent decode kernel and the LSE-combine + W_UV kernel.
+Default workload: the DeepSeek-V3 attention shape at 32K context (B=32,
+128 heads, r=512, rope 64, bf16), the shape the metric is quoted on.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle as the reference arm
+
+Prints ONE JSON line on rank 0. Under torchrun (N > 1) every rank decodes its
+own replica of the workload (the path shards over independent sequences:
+weak scaling, no collective on the data path); value = the cache bytes of all
+ranks / the slowest rank's time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+METRIC = "MLA decode: KV-cache GB/s & TFLOP/s vs B200 roofline; µs/step at 32K ctx"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="deepseek_v3")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05"], default="auto")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work of one step (measurement)
+# ----------------------------------------------------------------------------
+def step_work(wl, lens):
+    elt = 2 if wl.dtype == "bf16" else 4
+    B, Lq, H = len(lens), wl.q_len, wl.heads
+    r, dr, dn, dv, S = wl.latent_rank, wl.rope_dim, wl.nope_dim, wl.v_dim, wl.latent_shards
+    sum_l = int(sum(lens))
+    rows = H * Lq
+    cache = sum_l * (r + dr) * elt
+    q_full = B * rows * (r + dr) * elt
+    weights = H * dn * r * elt + H * r * dv * elt
+    io = B * rows * (dn + dr) * elt + B * rows * dv * elt
+    qk = 2 * rows * sum_l * (r + S * dr)
+    pv = 2 * rows * sum_l * r
+    absorb = 2 * B * rows * dn * r
+    upproj = 2 * B * rows * r * dv
+    return dict(cache_bytes=cache, step_bytes=cache + weights + io,
+                step_flops=qk + pv + absorb + upproj,
+                decode_bytes=cache + q_full, decode_flops=qk + pv,
+                exps=rows * sum_l * S)
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mla_latent_kv_21_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, kernel):
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(workload, {}).get(kernel)
+    if not ent or ent.get("source_digest") != kernel_source_digest():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.lines = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", self.gpu_id], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            rows.append((ts, parts))
+        inside = [p for ts, p in rows if t0 <= ts <= t1]
+        if not inside:
+            after = [p for ts, p in rows if ts >= t0]
+            inside = after[:1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[2]) for p in inside if num(p[2]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in inside:
+            for name, val in zip(names, p[6:10]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(inside[0][3]), "reasons": sorted(reasons),
+                "power_w_max": max((num(p[4]) or 0.0) for p in inside),
+                "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (one process per GPU)
+# ----------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+# ----------------------------------------------------------------------------
+# oracle timing (cpu_baseline and the reference arm)
+# ----------------------------------------------------------------------------
+def oracle_threads():
+    try:
+        import threadpoolctl
+        n = [i["num_threads"] for i in threadpoolctl.threadpool_info() if i["user_api"] == "blas"]
+        if n:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def time_oracle_sample(wl, inputs, pairs, tokens):
+    """Runs the oracle on (sequence, head) pairs over their first `tokens` keys
+    (Lq = 1 workloads) or full length; returns (seconds, outputs)."""
+    import numpy as np
+    from mla_workloads import logical_cache
+    from oracle import mla_oracle
+    qn = inputs["q_nope"].double().numpy()
+    qr = inputs["q_rope"].double().numpy()
+    wuk = inputs["w_uk"].double().numpy()
+    wuv = inputs["w_uv"].double().numpy()
+    outs = []
+    t0 = time.perf_counter()
+    for b, h in pairs:
+        c, k = logical_cache(inputs, b, wl)
+        n = min(tokens, c.shape[0]) if tokens else c.shape[0]
+        outs.append(mla_oracle.mla_decode(qn, qr, {b: c[:n].double().numpy()},
+                                          {b: k[:n].double().numpy()}, wuk, wuv,
+                                          wl.softmax_scale, wl.latent_shards, [b], [h]))
+    return time.perf_counter() - t0, outs
+
+
+def compare_sample(gpu_out, oracle_outs, pairs, dtype):
+    """max-abs / rel-Frobenius of the GPU output against the oracle's sampled rows."""
+    import numpy as np
+    got = np.concatenate([gpu_out[b, :, h].double().numpy().ravel() for b, h in pairs])
+    ref = np.concatenate([o[0, :, 0].ravel() for o in oracle_outs])
+    d = got - ref
+    return {"max_abs": float(np.abs(d).max()),
+            "rel_fro": float(np.linalg.norm(d) / np.linalg.norm(ref)),
+            "pairs": [list(p) for p in pairs],
+            "tolerance": ({"max_abs": 2e-2, "rel_fro": 5e-3} if dtype == "bf16"
+                          else {"rel_fro": 1e-5})}
+
+
+def reference_arm(args, wl, world, rank):
+    """The CPU oracle as it stands, timed on host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    from mla_workloads import generate
+    inputs = generate(wl)
+    lens = inputs["seq_lens"].tolist()
+    work = step_work(wl, lens)
+    B, H = len(lens), wl.heads
+    # calibrate: seconds per (head x token) on a small sample
+    t_cal, _ = time_oracle_sample(wl, inputs, [(0, 0)], 2048)
+    per_token = t_cal / 2048
+    budget = min(2.0, 150.0 / max(1, args.steps + args.warmup))
+    tokens = int(max(256, min(min(lens), budget / max(per_token, 1e-9))))
+    pairs = [(i % B, (7 * i) % H) for i in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        time_oracle_sample(wl, inputs, [pairs[i]], tokens)
+    total, done_tokens = 0.0, 0
+    for i in range(args.warmup, args.warmup + args.steps):
+        dt, _ = time_oracle_sample(wl, inputs, [pairs[i]], tokens)
+        total += dt
+        done_tokens += min(tokens, lens[pairs[i][0]])
+    frac = done_tokens / (sum(lens) * H)          # share of the step's (token, head) work
+    value = work["cache_bytes"] * frac / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": B, "heads": H, "q_len": wl.q_len,
+                   "context": wl.context, "latent_rank": wl.latent_rank,
+                   "rope_dim": wl.rope_dim, "latent_shards": wl.latent_shards},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step one (sequence, head) pair over its first "
+                                   f"{tokens} keys; throughput scaled by the pair's share "
+                                   f"of the step's (token x head) work"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    world, rank, local = dist_env()
+    from mla_workloads import WORKLOADS, generate
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        reference_arm(args, wl, world, rank)
+        return
+
+    import torch
+    import mla_latent_kv_21_b200 as M
+
+    dist = init_dist(world)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    peaks, peaks_kind = load_peaks()
+
+    inputs = generate(wl)
+    lens = inputs["seq_lens"].tolist()
+    work = step_work(wl, lens)
+    dev = {k: (v.to(device) if torch.is_tensor(v) else v) for k, v in inputs.items()}
+    kernel = {"auto": M.MLA_KERNEL_AUTO, "simt": M.MLA_KERNEL_SIMT,
+              "tcgen05": M.MLA_KERNEL_TCGEN05}[args.kernel]
+    dims = M.dims_for(wl.heads, wl.latent_rank, wl.rope_dim, wl.nope_dim, wl.v_dim, wl.q_len,
+                      wl.softmax_scale, wl.dtype, wl.latent_shards, wl.page_size)
+    plan = M.DecodePlan(dims, lens, kernel=kernel).allocate_workspace(device)
+    B = len(lens)
+    out = torch.empty((B, wl.q_len, wl.heads, wl.v_dim), dtype=wl.torch_dtype, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(events=None):
+        plan.run(dev["q_nope"], dev["q_rope"], dev["kv_pool"], dev["block_table"],
+                 dev["seq_lens"], dev["w_uk"], dev["w_uv"], out, stream.cuda_stream, events)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    status = plan.read_status()
+    if status != 0:
+        raise SystemExit(f"device status after warm-up: {M.mla_status_string(status)}")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    sampler.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    w0 = time.time()
+    t_start.record(stream)
+    for i in range(K):
+        step(ev[i])
+    t_stop.record(stream)
+    torch.cuda.synchronize(device)
+    w1 = time.time()
+    if dist:
+        dist.barrier()
+    sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_stop)
+    decode_ms = [a.elapsed_time(b) for a, b in ev]
+    if dist:
+        t = torch.tensor([elapsed_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    status = plan.read_status()
+    if status != 0:
+        raise SystemExit(f"device status after timing: {M.mla_status_string(status)}")
+
+    # ---- end to end through the public API: host buffers, copies in the timed region
+    host = {k: inputs[k].pin_memory() for k in ("q_nope", "q_rope", "block_table", "seq_lens")}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    Ke = max(1, min(K, 50))
+
+    def e2e_step():
+        for k, t in host.items():
+            dev[k].copy_(t, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    ms_step = elapsed_ms / K
+    value = world * work["cache_bytes"] / (ms_step * 1e-3) / 1e9
+    e2e_value = world * work["cache_bytes"] / (e2e_ms / Ke * 1e-3) / 1e9
+    info = plan.info
+    kname = "tcgen05" if info.kernel == M.MLA_KERNEL_TCGEN05 else "simt"
+    dec_s = statistics.mean(decode_ms) * 1e-3
+    hbm_peak = peaks["hbm_gbs"]
+    if kname == "tcgen05":
+        flop_peak = peaks["bf16_tflops"]
+        flop_kind = "bf16 tensor"
+    else:
+        # CUDA-core fp32 FMA: 148 SMs x 128 lanes x 2 flops x max SM clock
+        flop_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        flop_kind = "fp32 FMA (ALU)"
+    t_bytes = work["decode_bytes"] / (hbm_peak * 1e9)
+    t_flops = work["decode_flops"] / (flop_peak * 1e12)
+    if t_bytes >= t_flops:
+        roof = {"bound": "hbm", "achieved": work["decode_bytes"] / dec_s / 1e9, "peak": hbm_peak,
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor" if kname == "tcgen05" else "alu",
+                "achieved": work["decode_flops"] / dec_s / 1e12, "peak": flop_peak,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic(wl.name, kname)
+    roof["kernel"] = f"decode_{kname}"
+    roof["peak_source"] = f"{peaks_kind} ({flop_kind} for FLOPs)"
+    roof["decode_us"] = dec_s * 1e6
+    step_roof_s = max(work["step_bytes"] / (hbm_peak * 1e9),
+                      work["step_flops"] / (peaks["bf16_tflops"] * 1e12))
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "batch": B, "heads": wl.heads, "q_len": wl.q_len,
+                   "context": wl.context, "latent_rank": wl.latent_rank,
+                   "rope_dim": wl.rope_dim, "nope_dim": wl.nope_dim, "v_dim": wl.v_dim,
+                   "latent_shards": wl.latent_shards, "page_size": wl.page_size,
+                   "kernel": kname, "workers": info.num_workers,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"inputs larger than L2 (cache {work['cache_bytes'] / 1e9:.2f} GB)"},
+        "us_per_step": ms_step * 1e3,
+        "tflops": work["step_flops"] / (ms_step * 1e-3) / 1e12,
+        "step_roofline_us": step_roof_s * 1e6,
+        "step_roofline_frac": step_roof_s / (ms_step * 1e-3),
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "us_per_step": e2e_ms / Ke * 1e3, "steps": Ke},
+        "gpu_launches": info.launches_per_run * K,
+        "clocks": sampler.summary(w0, w1),
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the oracle as it stands on the host cores, bounded sample; its sampled
+        # outputs double as a parity spot check of this run's GPU output
+        pairs = [(0, 0), (B // 2, wl.heads // 3), (B - 1, wl.heads - 1)]
+        dt, outs = time_oracle_sample(wl, inputs, pairs, 0)
+        done = sum(lens[b] for b, _ in pairs)
+        frac = done / (sum(lens) * wl.heads)
+        line["cpu_baseline"] = {
+            "value": work["cache_bytes"] * frac / dt / 1e9, "unit": "GB/s",
+            "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{len(pairs)} (sequence, head) pairs at full length, fp64 numpy, "
+                      f"scaled by their share of the step's (token x head) work; {dt:.1f} s"}
+        line["parity_sample"] = compare_sample(out.cpu(), outs, pairs, wl.dtype)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,189 @@
+/*
+ * mla_decode.h — C ABI of the B200 (sm_100a) MLA latent-cache decode library.
+ *
+ * One call of mla_decode_run performs one decode step of Multi-Head Latent
+ * Attention in its absorbed form over a paged latent KV cache:
+ *
+ *   q_lat[b,t,h,:] = q_nope[b,t,h,:] . W_UK[h]                      (absorb)
+ *   s[j]   = scale * (q_lat . cKV[b,j] + q_rope[b,t,h] . k_rope[b,j]),  j <= L_b - Lq + t
+ *   o_lat  = softmax(s) . cKV[b, :]                                  (latent accumulation)
+ *   out[b,t,h,:] = o_lat . W_UV[h]                                   (up-projection)
+ *
+ * Sources: the TPLA abstract (latent cKV cache; partition of the latent and of
+ * each head's input dimension, independent attention per shard, summed
+ * results), "TransMLA: Multi-Head Latent Attention Is All You Need" abstract
+ * (the Absorb operation keeps the cache compressed), the pith.science verdict
+ * record for 2502.07864 (key_machinery: absorbed form is exact; core_discovery:
+ * one shared multi-query RoPE key; referee report on Eq. 26: the MQA form).
+ *
+ * Layouts (row-major, last dimension contiguous, element type = dims.dtype):
+ *   q_nope   [B, Lq, H, d_nope]
+ *   q_rope   [B, Lq, H, d_rope]   query after RoPE (decode applies no rotation)
+ *   kv_cache [num_blocks, page_size, r + d_rope]; columns [0, r) are cKV,
+ *            columns [r, r + d_rope) the decoupled RoPE key (after RoPE)
+ *   block_table int32 [B, block_table_stride]; entry (b, i) is the block that
+ *            holds tokens [i*page_size, (i+1)*page_size) of sequence b
+ *   seq_lens int32 [B], L_b counts the Lq query tokens (they are the newest
+ *            Lq cache rows; query t sees keys j <= L_b - Lq + t)
+ *   w_uk     [H, d_nope, r]     w_uv [H, r, d_v]
+ *   out      [B, Lq, H, d_v]
+ * TPLA (latent_shards = S > 1): shard s owns latent columns
+ * [s*r/S, (s+1)*r/S) of cKV, of W_UK[h] and of W_UV[h]; every shard adds the
+ * full RoPE score and has its own softmax; the shard outputs are summed.
+ *
+ * Ownership: the caller owns every device buffer, including the workspace;
+ * the library owns only the plan (host memory). mla_decode_run does not
+ * allocate, synchronise or read device memory on the host, so a stream may be
+ * captured into a CUDA graph around it.
+ *
+ * Errors: every call returns an mla_status_t; nothing aborts the process and
+ * no exception crosses the ABI. Errors found on the device (a block-table
+ * entry outside [0, num_blocks), a sequence length outside
+ * [Lq, block_table_stride * page_size], a bounded wait that ran out) are
+ * recorded in a status word inside the workspace; the affected work is
+ * skipped (never read out of bounds) and mla_decode_read_status returns the
+ * first recorded code.
+ */
+#ifndef MLA_DECODE_H
+#define MLA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_ABI_VERSION 1
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,         /* null pointer, non-positive size, bad length */
+  MLA_ERR_UNSUPPORTED = 2,         /* dims outside what the kernels implement */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes below the plan's size */
+  MLA_ERR_CUDA = 4,                /* a CUDA runtime call failed */
+  MLA_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device-side wait ran out */
+  MLA_ERR_BOUNDS = 6,              /* block id or sequence length out of range */
+  MLA_ERR_NO_DEVICE = 7            /* no usable sm_100 device */
+} mla_status_t;
+
+typedef enum { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype_t;
+
+/* Kernel family selection (mla_plan_options_t.kernel). */
+typedef enum {
+  MLA_KERNEL_AUTO = 0,    /* tcgen05 path where supported, else SIMT */
+  MLA_KERNEL_SIMT = 1,    /* CUDA-core fp32 path (all dims; the fp32 path) */
+  MLA_KERNEL_TCGEN05 = 2  /* tensor-core path: bf16, r = 512, d_rope = 64, H*Lq <= 128 */
+} mla_kernel_t;
+
+typedef struct {
+  int32_t num_heads;      /* H */
+  int32_t latent_rank;    /* r (cKV width) */
+  int32_t rope_dim;       /* d_rope */
+  int32_t nope_dim;       /* d_nope (W_UK rows per head) */
+  int32_t v_dim;          /* d_v (W_UV columns per head) */
+  int32_t q_len;          /* Lq query tokens per sequence (1, or 2 for MTP) */
+  int32_t page_size;      /* tokens per cache block; 64 */
+  int32_t latent_shards;  /* 1 = MLA, 2 = TPLA two-shard form */
+  float softmax_scale;    /* multiplies q.k; usually 1/sqrt(d_nope + d_rope) */
+  int32_t dtype;          /* mla_dtype_t of every tensor argument */
+} mla_dims_t;
+
+typedef struct {
+  int32_t num_sms;        /* SMs to plan for; 0 = query the current device */
+  int32_t kernel;         /* mla_kernel_t */
+  int32_t num_workers;    /* 0 = automatic; else the number of page ranges */
+} mla_plan_options_t;
+
+typedef struct {
+  int32_t batch;
+  int32_t rows;             /* H * Lq rows per sequence */
+  int32_t kernel;           /* mla_kernel_t that mla_decode_run launches */
+  int32_t num_workers;      /* page ranges (one CTA pair each on tcgen05) */
+  int32_t num_split_slots;  /* partial-result slots = num_workers + batch - 1 */
+  int32_t launches_per_run; /* kernels one mla_decode_run launches */
+  int64_t total_pages;      /* sum over b of ceil(L_b / page_size) at plan time */
+  uint64_t workspace_bytes;
+} mla_plan_info_t;
+
+typedef struct mla_plan* mla_plan_t; /* opaque, library-owned host object */
+
+/* Supported-dims check and workspace sizing for a batch.
+ * seq_lens_host [batch] (host memory) gives the lengths the plan balances;
+ * the device lengths passed to run may differ as long as each stays in
+ * [Lq, block_table_stride * page_size]: the split partition is recomputed
+ * on the device every run, so only balance (not correctness) depends on the
+ * plan-time lengths. On success *plan_out receives a new plan (free it with
+ * mla_plan_destroy) and *workspace_bytes the workspace size run needs. */
+mla_status_t mla_decode_plan(const mla_dims_t* dims, int32_t batch,
+                             const int32_t* seq_lens_host, int32_t num_sms,
+                             mla_plan_t* plan_out, size_t* workspace_bytes);
+
+/* mla_decode_plan with explicit options (kernel family, worker count);
+ * opts may be NULL for the defaults. */
+mla_status_t mla_decode_plan_ex(const mla_dims_t* dims, int32_t batch,
+                                const int32_t* seq_lens_host,
+                                const mla_plan_options_t* opts,
+                                mla_plan_t* plan_out, size_t* workspace_bytes);
+
+/* One decode step, enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ * stream). All pointers are device pointers except `plan`. The workspace must
+ * hold at least the plan's workspace_bytes and may not be shared by two runs
+ * in flight at once. Returns MLA_OK once the kernels are enqueued. */
+mla_status_t mla_decode_run(mla_plan_t plan,
+                            const void* q_nope, const void* q_rope,
+                            const void* kv_cache, int64_t num_blocks,
+                            const int32_t* block_table, int32_t block_table_stride,
+                            const int32_t* seq_lens_dev,
+                            const void* w_uk, const void* w_uv,
+                            void* out, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Options of mla_decode_run_ex. */
+typedef struct {
+  /* cudaEvent_t handles recorded on `stream` immediately before and after the
+   * split-KV decode kernel (the dominant kernel of a run), for timing it
+   * inside a full step; NULL to record nothing. The events are caller-owned. */
+  void* decode_start_event;
+  void* decode_stop_event;
+} mla_run_options_t;
+
+/* mla_decode_run with options; opts may be NULL (then identical to run). */
+mla_status_t mla_decode_run_ex(mla_plan_t plan,
+                               const void* q_nope, const void* q_rope,
+                               const void* kv_cache, int64_t num_blocks,
+                               const int32_t* block_table, int32_t block_table_stride,
+                               const int32_t* seq_lens_dev,
+                               const void* w_uk, const void* w_uv,
+                               void* out, void* workspace, size_t workspace_bytes,
+                               void* stream, const mla_run_options_t* opts);
+
+/* Clears the workspace header (status word) with an async memset on `stream`.
+ * Call once after allocating a workspace, before its first run. */
+mla_status_t mla_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, copies the workspace status word to *device_status
+ * (an mla_status_t value; MLA_OK if nothing was recorded) and clears it. */
+mla_status_t mla_decode_read_status(const void* workspace, void* stream,
+                                    int32_t* device_status);
+
+/* Plan facts for callers and tests. */
+mla_status_t mla_plan_get_info(mla_plan_t plan, mla_plan_info_t* info);
+
+/* The plan-time split partition, computed on the host by the same function the
+ * kernels evaluate on the device. Each segment is 5 int32 values:
+ * (worker, sequence, first page, end page (exclusive), partial slot).
+ * Writes min(capacity, count) segments to `out` (may be NULL when capacity is
+ * 0) and the total number to *count. */
+mla_status_t mla_plan_segments(mla_plan_t plan, int32_t* out, int64_t capacity,
+                               int64_t* count);
+
+void mla_plan_destroy(mla_plan_t plan);
+const char* mla_status_string(mla_status_t status);
+int32_t mla_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H */

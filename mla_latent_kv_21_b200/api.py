@@ -1,0 +1,76 @@
+"""Torch-tensor convenience over the C ABI (marshalling only: every step of the
+decode runs inside libmla_decode.so; torch provides device memory and streams)."""
+
+from __future__ import annotations
+
+from typing import Optional, Sequence
+
+from . import _lib as L
+
+
+def dims_for(heads: int, latent_rank: int, rope_dim: int, nope_dim: int, v_dim: int,
+             q_len: int, softmax_scale: float, dtype: str = "bf16", latent_shards: int = 1,
+             page_size: int = 64) -> L.mla_dims_t:
+    return L.make_dims(heads, latent_rank, rope_dim, nope_dim, v_dim, q_len, page_size,
+                       latent_shards, float(softmax_scale),
+                       L.MLA_BF16 if dtype == "bf16" else L.MLA_FP32)
+
+
+class DecodePlan:
+    """Owns one plan handle and (once bound) its device workspace tensor."""
+
+    def __init__(self, dims: L.mla_dims_t, seq_lens_host: Sequence[int], num_sms: int = 0,
+                 kernel: int = L.MLA_KERNEL_AUTO, num_workers: int = 0):
+        self.dims = dims
+        self.handle, self.workspace_bytes = L.mla_decode_plan_ex(
+            dims, list(seq_lens_host), num_sms, kernel, num_workers)
+        self.info = L.mla_plan_get_info(self.handle)
+        self.workspace = None
+
+    def allocate_workspace(self, device) -> "DecodePlan":
+        import torch
+        self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=device)
+        L.mla_workspace_init(self.workspace.data_ptr(), self.workspace_bytes,
+                             torch.cuda.current_stream(device).cuda_stream)
+        return self
+
+    def segments(self):
+        return L.mla_plan_segments(self.handle)
+
+    def run(self, q_nope, q_rope, kv_pool, block_table, seq_lens, w_uk, w_uv, out,
+            stream: Optional[int] = None, decode_events=None) -> None:
+        """All arguments are device tensors laid out as in include/mla_decode.h."""
+        import torch
+        if self.workspace is None:
+            self.allocate_workspace(q_nope.device)
+        for name, t in (("q_nope", q_nope), ("q_rope", q_rope), ("kv_pool", kv_pool),
+                        ("block_table", block_table), ("seq_lens", seq_lens), ("w_uk", w_uk),
+                        ("w_uv", w_uv), ("out", out)):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if stream is None:
+            stream = torch.cuda.current_stream(q_nope.device).cuda_stream
+        ev0, ev1 = (None, None) if decode_events is None else (
+            decode_events[0].cuda_event, decode_events[1].cuda_event)
+        L.mla_decode_run_ex(self.handle, q_nope.data_ptr(), q_rope.data_ptr(),
+                            kv_pool.data_ptr(), kv_pool.shape[0], block_table.data_ptr(),
+                            block_table.shape[1], seq_lens.data_ptr(), w_uk.data_ptr(),
+                            w_uv.data_ptr(), out.data_ptr(), self.workspace.data_ptr(),
+                            self.workspace_bytes, stream, ev0, ev1)
+
+    def read_status(self, stream: Optional[int] = None) -> int:
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream(self.workspace.device).cuda_stream
+        return L.mla_decode_read_status(self.workspace.data_ptr(), stream)
+
+    def close(self) -> None:
+        if self.handle:
+            L.mla_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

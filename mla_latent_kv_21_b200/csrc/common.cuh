@@ -1,0 +1,118 @@
+// Shared definitions of the decode library: the split partition (evaluated
+// identically by the host plan and by every kernel), the workspace layout and
+// the kernel parameter block.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/mla_decode.h"
+
+#define MLA_HD __host__ __device__ __forceinline__
+
+namespace mla {
+
+// ---------------------------------------------------------------------------
+// Split partition.
+//
+// The pages of all sequences are concatenated (sequence b owns global pages
+// [cum[b], cum[b+1]), cum[b] = sum_{i<b} ceil(L_i / P)) and cut into W
+// contiguous page ranges, worker w owning [start(w), start(w+1)) with
+// start(w) = floor(w * G / W). A worker's range meets one or more sequences;
+// each (worker, sequence) intersection is one split segment whose partial
+// result goes to slot w + b. Along the concatenated page order both w and b
+// are non-decreasing and at least one of them grows from one segment to the
+// next, so w + b is strictly increasing: slots are unique, and W + B - 1 slots
+// always suffice whatever the lengths are.
+// ---------------------------------------------------------------------------
+MLA_HD int64_t worker_page_start(int64_t w, int64_t G, int64_t W) {
+  return (w * G) / W;
+}
+
+// The worker whose range holds global page x (0 <= x < G): the largest w with
+// start(w) <= x, i.e. w = ceil((x + 1) * W / G) - 1, clamped to W - 1.
+MLA_HD int64_t page_owner(int64_t x, int64_t G, int64_t W) {
+  int64_t w = ((x + 1) * W + G - 1) / G - 1;
+  return w < W - 1 ? w : W - 1;
+}
+
+MLA_HD int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------------------
+// Workspace layout (byte offsets from the workspace base; all 1 KiB aligned).
+//   [0]            int32 status word (first device-side error, sticky)
+//   [4]            int32 lengths_ok (written by the first kernel of a run)
+//   cum            int64 [B + 1] page prefix sums of this run's seq_lens
+//   q              [B * Lq * H, r + d_rope] absorbed query rows (dims.dtype)
+//   o_part         fp32 [slots, rows, r]  per-segment O_lat / l
+//   lse_part       fp32 [slots, rows, S]  per-segment log2-sum-exp per shard
+// ---------------------------------------------------------------------------
+struct WorkspaceLayout {
+  size_t cum, q, o_part, lse_part, total;
+};
+
+MLA_HD size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WorkspaceLayout workspace_layout(int64_t B, int64_t Lq, int64_t H, int64_t r,
+                                        int64_t dr, int64_t shards, int64_t elt_bytes,
+                                        int64_t slots) {
+  WorkspaceLayout L{};
+  size_t off = 1024;
+  L.cum = off;
+  off = align_up(off + sizeof(int64_t) * (B + 1), 1024);
+  L.q = off;
+  off = align_up(off + (size_t)(B * Lq * H) * (r + dr) * elt_bytes, 1024);
+  L.o_part = off;
+  off = align_up(off + (size_t)slots * (Lq * H) * r * sizeof(float), 1024);
+  L.lse_part = off;
+  off = align_up(off + (size_t)slots * (Lq * H) * shards * sizeof(float), 1024);
+  L.total = off;
+  return L;
+}
+
+// Finite stand-in for log(0): a segment row that saw no key.
+constexpr float kEmptyLse = -1.0e30f;
+
+// ---------------------------------------------------------------------------
+// Parameters shared by the kernels of one run.
+// ---------------------------------------------------------------------------
+struct RunParams {
+  // inputs
+  const void* q_nope;
+  const void* q_rope;
+  const void* kv;          // pool
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const void* w_uk;
+  const void* w_uv;
+  void* out;
+  // workspace
+  int32_t* status;
+  int32_t* lengths_ok;
+  int64_t* cum;
+  void* q;                 // absorbed query rows
+  float* o_part;
+  float* lse_part;
+  // sizes
+  int64_t num_blocks;
+  int32_t bt_stride;
+  int32_t B, Lq, H, r, dr, dn, dv, P, S;
+  int32_t rows;            // H * Lq
+  int32_t W;               // workers
+  float scale_log2;        // softmax_scale * log2(e)
+};
+
+__device__ __forceinline__ void record_error(int32_t* status, int32_t code) {
+  atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_float(float x);
+template <> __device__ __forceinline__ float from_float<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+}  // namespace mla

@@ -1,0 +1,147 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads and
+exports every declared symbol, argument validation, and the split partition
+against an independent recomputation (integer-exact)."""
+
+import os
+import random
+import re
+import subprocess
+
+import pytest
+
+import mla_latent_kv_21_b200 as M
+from mla_latent_kv_21_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if fn.endswith(".h"):
+            text = open(os.path.join(inc, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names.update(re.findall(r"\b(mla_[a-z_0-9]+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_functions()
+    assert declared, "no declarations found"
+    out = subprocess.run(["nm", "-D", "--defined-only", M.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\b[TW]\s+(mla_\w+)", out))
+    assert declared <= exported, declared - exported
+    assert declared == set(L.EXPORTED)
+    assert L.mla_abi_version() == 1
+
+
+def _dims(**kw):
+    d = dict(heads=128, latent_rank=512, rope_dim=64, nope_dim=128, v_dim=128, q_len=1,
+             softmax_scale=192 ** -0.5, dtype="bf16", latent_shards=1)
+    d.update(kw)
+    return M.dims_for(**d)
+
+
+def test_status_strings():
+    for s in range(8):
+        assert L.mla_status_string(s) and L.mla_status_string(s) != "unknown status"
+    assert L.mla_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(heads=0), L.MLA_ERR_INVALID_ARG),
+    (dict(softmax_scale=float("nan")), L.MLA_ERR_INVALID_ARG),
+    (dict(page_size=32), L.MLA_ERR_UNSUPPORTED),
+    (dict(latent_shards=3), L.MLA_ERR_UNSUPPORTED),
+    (dict(latent_rank=1024), L.MLA_ERR_UNSUPPORTED),
+    (dict(nope_dim=256), L.MLA_ERR_UNSUPPORTED),
+])
+def test_plan_rejects_bad_dims(kw, status):
+    with pytest.raises(L.MlaError) as e:
+        L.mla_decode_plan(_dims(**kw), [100, 200], num_sms=148)
+    assert e.value.status == status
+
+
+def test_plan_rejects_short_sequences():
+    with pytest.raises(L.MlaError) as e:
+        L.mla_decode_plan(_dims(q_len=2), [5, 1], num_sms=148)
+    assert e.value.status == L.MLA_ERR_INVALID_ARG
+
+
+def test_run_rejects_null_and_small_workspace():
+    plan, ws = L.mla_decode_plan_ex(_dims(), [100], num_sms=148, kernel=L.MLA_KERNEL_SIMT)
+    try:
+        with pytest.raises(L.MlaError) as e:
+            L.mla_decode_run(plan, 0, 0, 0, 1, 0, 1, 0, 0, 0, 0, 0, ws, 0)
+        assert e.value.status == L.MLA_ERR_INVALID_ARG
+        fake = 1 << 20  # never dereferenced: the size check comes first
+        with pytest.raises(L.MlaError) as e:
+            L.mla_decode_run(plan, fake, fake, fake, 1, fake, 2, fake, fake, fake, fake, fake,
+                             ws - 1, 0)
+        assert e.value.status == L.MLA_ERR_WORKSPACE_TOO_SMALL
+    finally:
+        L.mla_plan_destroy(plan)
+
+
+def _reference_segments(lens, P, W):
+    """Independent recomputation of the split partition."""
+    pages = [-(-x // P) for x in lens]
+    bounds = [0]
+    for n in pages:
+        bounds.append(bounds[-1] + n)
+    G = bounds[-1]
+    segs = []
+    for w in range(W):
+        a, e = w * G // W, (w + 1) * G // W
+        for b in range(len(lens)):
+            lo, hi = max(a, bounds[b]), min(e, bounds[b + 1])
+            if lo < hi:
+                segs.append((w, b, lo - bounds[b], hi - bounds[b], w + b))
+    return segs, pages
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_split_partition_matches_independent_recomputation(seed):
+    rng = random.Random(seed)
+    B = rng.choice([1, 2, 3, 7, 32, 64])
+    q_len = rng.choice([1, 2])
+    lens = [rng.randint(q_len, rng.choice([64, 65, 300, 5000, 32768])) for _ in range(B)]
+    kernel = rng.choice([L.MLA_KERNEL_SIMT, L.MLA_KERNEL_AUTO])
+    workers = rng.choice([0, 0, 1, 5, 74, 1000])
+    plan, ws = L.mla_decode_plan_ex(_dims(q_len=q_len), lens, num_sms=148, kernel=kernel,
+                                    num_workers=workers)
+    try:
+        info = L.mla_plan_get_info(plan)
+        W = info.num_workers
+        got = L.mla_plan_segments(plan)
+        want, pages = _reference_segments(lens, 64, W)
+        assert got == want
+        assert info.total_pages == sum(pages)
+        assert 1 <= W <= sum(pages)
+        assert info.num_split_slots == W + B - 1
+        # each sequence covered exactly once, in order, by its segments
+        for b in range(B):
+            mine = [s for s in got if s[1] == b]
+            assert mine[0][2] == 0 and mine[-1][3] == pages[b]
+            for s0, s1 in zip(mine, mine[1:]):
+                assert s0[3] == s1[2]
+        slots = [s[4] for s in got]
+        assert len(set(slots)) == len(slots) and max(slots) < W + B - 1
+        assert slots == sorted(slots)
+        assert ws == info.workspace_bytes
+    finally:
+        L.mla_plan_destroy(plan)
+
+
+def test_workspace_holds_partials_for_every_slot():
+    lens = [32768] * 32
+    plan, ws = L.mla_decode_plan_ex(_dims(), lens, num_sms=148, kernel=L.MLA_KERNEL_SIMT)
+    try:
+        info = L.mla_plan_get_info(plan)
+        rows, slots = 128, info.num_split_slots
+        need = slots * rows * 512 * 4 + slots * rows * 4 + 32 * 128 * 576 * 2 + 33 * 8
+        assert ws >= need
+    finally:
+        L.mla_plan_destroy(plan)
