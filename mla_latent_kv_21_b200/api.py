@@ -50,8 +50,8 @@ class DecodePlan:
                 raise ValueError(f"{name} must be a contiguous CUDA tensor")
         if stream is None:
             stream = torch.cuda.current_stream(q_nope.device).cuda_stream
-        ev0, ev1 = (None, None) if decode_events is None else (
-            decode_events[0].cuda_event, decode_events[1].cuda_event)
+        # decode_events: optional (start, stop) raw cudaEvent_t handles (ints)
+        ev0, ev1 = (None, None) if decode_events is None else decode_events
         L.mla_decode_run_ex(self.handle, q_nope.data_ptr(), q_rope.data_ptr(),
                             kv_pool.data_ptr(), kv_pool.shape[0], block_table.data_ptr(),
                             block_table.shape[1], seq_lens.data_ptr(), w_uk.data_ptr(),

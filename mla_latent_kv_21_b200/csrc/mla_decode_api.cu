@@ -101,8 +101,8 @@ mla_status_t mla_decode_plan_ex(const mla_dims_t* dims, int32_t batch, const int
   if (o.num_workers > 0) {
     W = o.num_workers;
   } else if (kernel == MLA_KERNEL_TCGEN05) {
-    // one CTA pair per worker; at least two pages (one pair step) each
-    W = std::max<int64_t>(1, std::min<int64_t>(sms / 2, G / 2));
+    // one CTA pair per worker (a cluster of two SMs); a pair step is one page
+    W = std::max<int64_t>(1, std::min<int64_t>(sms / 2, G));
   } else {
     W = std::max<int64_t>(1, std::min<int64_t>(sms, G));
   }
