@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--workload", default="deepseek_v3")
     ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05"], default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling cases)")
+    ap.add_argument("--context", type=int, default=0, help="override every length (profiling cases)")
     return ap.parse_args()
 
 
@@ -328,6 +330,10 @@ def main():
     world, rank, local = dist_env()
     from mla_workloads import WORKLOADS, generate
     wl = WORKLOADS[args.workload]
+    if args.batch:
+        wl = wl.with_(batch=args.batch)
+    if args.context:
+        wl = wl.with_(context=args.context, context_min=0)
     if args.impl == "reference":
         reference_arm(args, wl, world, rank)
         return

@@ -284,4 +284,13 @@ mla_status_t mla_decode_read_status(const void* workspace, void* stream_, int32_
   return MLA_OK;
 }
 
+#ifdef MLA_TRACE
+// Debug builds only: copies the event trace (see tc_decode.cuh) to host memory.
+int mla_debug_trace_read(unsigned long long* host, size_t n) {
+  const size_t cap = sizeof(tc::g_trace) / sizeof(unsigned long long);
+  if (n > cap) n = cap;
+  return cudaMemcpyFromSymbol(host, tc::g_trace, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 1;
+}
+#endif
+
 }  // extern "C"

@@ -58,6 +58,12 @@ __device__ __forceinline__ void mbar_arrive_local(uint32_t bar) {
                :: "r"(bar) : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive_expect_tx_local(uint32_t bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\t"
+               "mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 st, [%0], %1;\n\t}"
+               :: "r"(bar), "r"(bytes) : "memory");
+}
+
 // Arrive on a barrier anywhere in the cluster (bar = shared::cluster address).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
@@ -79,12 +85,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
+// CTA-scope acquire: enough for barriers completed by tcgen05.commit or by
+// arrivals from threads of this CTA.
+__device__ __forceinline__ bool mbar_try_wait_cta(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity to complete. kCluster
+// selects cluster-scope acquire (arrivals from the peer CTA's threads).
+template <bool kCluster = true>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto probe = [&]() { return kCluster ? mbar_try_wait(bar, parity) : mbar_try_wait_cta(bar, parity); };
+  if (probe()) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (probe()) return true;
     if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
   }
 }

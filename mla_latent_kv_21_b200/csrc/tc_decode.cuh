@@ -86,9 +86,24 @@ enum : int {
   B_COUNT = 23
 };
 
-struct TcParams {
-  RunParams p;
-};
+// Optional event trace (compile with -DMLA_TRACE): SM clock of each role's
+// per-step events for the first kTraceWorkers workers, read back on the host
+// with mla_debug_trace_read(). Off in normal builds.
+#ifdef MLA_TRACE
+constexpr int kTraceWorkers = 4, kTraceKinds = 8, kTraceSteps = 64;
+__device__ unsigned long long g_trace[kTraceWorkers * 2 * kTraceKinds * kTraceSteps];
+#define MLA_TRACE_EV(w, rank, kind, step)                                                \
+  do {                                                                                   \
+    if ((w) < kTraceWorkers && (step) < kTraceSteps) {                                   \
+      unsigned long long t_;                                                             \
+      asm volatile("mov.u64 %0, %%clock64;" : "=l"(t_));                                 \
+      g_trace[(((w) * 2 + (rank)) * kTraceKinds + (kind)) * kTraceSteps + (step)] = t_;   \
+    }                                                                                    \
+  } while (0)
+#else
+#define MLA_TRACE_EV(w, rank, kind, step) do {} while (0)
+#endif
+enum { EV_LOAD = 0, EV_RELOAD, EV_QK, EV_PV, EV_S_READY, EV_P_DONE, EV_PBUF_FREE, EV_PV_READY };
 
 // Walks the worker's split segments: calls f(seg_index, b, first_page, end_page).
 template <typename F>
@@ -108,6 +123,39 @@ __device__ __forceinline__ void for_each_segment(const RunParams& p, int w, F&& 
     if (!f(seg, b, (int)pb, (int)pe)) return;
   }
 }
+
+// Sequential walk over the worker's steps (one page each): sequence b, page
+// within the sequence, end page of the segment, first-of-segment flag.
+struct StepCursor {
+  int b, page, pe;
+  bool first;
+  int64_t g1;
+  // returns the number of steps of worker w
+  __device__ __forceinline__ int init(const RunParams& p, int w) {
+    const int64_t G = p.cum[p.B];
+    const int64_t g0 = worker_page_start(w, G, p.W);
+    g1 = worker_page_start(w + 1, G, p.W);
+    int lo = 0, hi = p.B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.cum[mid] <= g0) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    page = (int)(g0 - p.cum[b]);
+    pe = (int)(min(p.cum[b + 1], g1) - p.cum[b]);
+    first = true;
+    return (int)(g1 - g0);
+  }
+  __device__ __forceinline__ void next(const RunParams& p) {
+    first = false;
+    if (++page >= pe && b + 1 < p.B && p.cum[b + 1] < g1) {
+      ++b;
+      page = 0;
+      pe = (int)(min(p.cum[b + 1], g1) - p.cum[b]);
+      first = true;
+    }
+  }
+};
 
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk16) {
   return row * 128 + ((chunk16 ^ (row & 7)) << 4);
@@ -130,6 +178,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto bar = [&](int i) -> uint32_t { return base + L::bars + 8u * i; };
   auto leader_bar = [&](int i) -> uint32_t { return map_to_cta(bar(i), 0); };
+  // arrival on a leader-owned barrier: CTA-local release on the leader itself
+  auto arrive_leader = [&](int i) {
+    if (rank == 0) mbar_arrive_local(bar(i)); else mbar_arrive_cluster(leader_bar(i));
+  };
+  auto expect_leader = [&](int i, uint32_t bytes) {
+    if (rank == 0) mbar_arrive_expect_tx_local(bar(i), bytes);
+    else mbar_arrive_expect_tx_cluster(leader_bar(i), bytes);
+  };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::misc + 8);
   float* xch = reinterpret_cast<float*>(gbase + L::xch);
@@ -160,88 +216,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_kv);
       prefetch_tmap(&tm_q);
-      // Flat list of steps: (segment, b, page). Loads run two steps ahead of
-      // the V re-reads; Q is (re)loaded at each segment start once the previous
-      // segment's QK MMAs are done with it.
-      int nsteps = 0;
-      for_each_segment(p, w, [&](int, int, int pb, int pe) { nsteps += pe - pb; return true; });
-      // step -> (b, page, first-of-segment) is recomputed by scanning segments
-      auto step_info = [&](int target, int& b_out, int& page_out, bool& first_out) {
-        int i = 0;
-        for_each_segment(p, w, [&](int, int b, int pb, int pe) {
-          if (target < i + (pe - pb)) {
-            b_out = b;
-            page_out = pb + (target - i);
-            first_out = target == i;
-            return false;
-          }
-          i += pe - pb;
-          return true;
-        });
-      };
-      auto block_of = [&](int b, int page) -> int32_t {
-        int32_t blk = p.block_table[(int64_t)b * p.bt_stride + page];
+      // The worker's pages, in order, are its steps. Loads run two steps ahead
+      // of the V re-reads; Q is (re)loaded at each segment start once the
+      // previous segment's QK MMAs are done with it. Two sequential cursors
+      // walk the steps; the block id of each stage is kept for its re-read.
+      StepCursor ld, rl;
+      const int nsteps = ld.init(p, w);
+      rl.init(p, w);
+      int32_t stage_blk[kStages] = {0, 0, 0};
+      auto block_of = [&](const StepCursor& c) -> int32_t {
+        int32_t blk = p.block_table[(int64_t)c.b * p.bt_stride + c.page];
         if (blk < 0 || blk >= p.num_blocks) {
           record_error(p.status, MLA_ERR_BOUNDS);
-          blk = 0;  // in-bounds stand-in; the softmax masks the page
+          blk = 0;  // in-bounds stand-in; the result is flagged by the status word
         }
         return blk;
       };
-      int seg_count = 0;
-      auto load_step = [&](int i) -> bool {
-        int b = 0, page = 0;
-        bool first = false;
-        step_info(i, b, page, first);
-        if (first) {
+      auto load_step = [&](int i, int32_t blk) -> bool {
+        if (ld.first) {
           if (i > 0) {
             // previous segment's last QK must be done before Q is overwritten
             const int j = i - 1;
-            if (!mbar_wait(bar(B_QK_DONE + j % kStages), (j / kStages) & 1)) return false;
+            if (!mbar_wait<false>(bar(B_QK_DONE + j % kStages), (j / kStages) & 1)) return false;
           }
           const uint32_t qb = leader_bar(B_Q_FULL);
-          mbar_arrive_expect_tx_cluster(qb, kQBytes);
-          const int y = b * p.rows + 64 * (int)rank;
+          expect_leader(B_Q_FULL, kQBytes);
+          const int y = ld.b * p.rows + 64 * (int)rank;
           for (int k = 0; k < kChunks; ++k)
             tma_load_2d_pair(base + L::q + k * kQChunkBytes, &tm_q, 64 * k, y, qb);
-          ++seg_count;
         }
         const int st = i % kStages;
-        const int32_t blk = block_of(b, page);
+        stage_blk[st] = blk;
         const uint32_t kb = leader_bar(B_KV_FULL + st);
-        mbar_arrive_expect_tx_cluster(kb, kStageBytes);
+        expect_leader(B_KV_FULL + st, kStageBytes);
         const int y = blk * 64 + 32 * (int)rank;
         const uint32_t sb = base + L::kv + st * kStageBytes;
         for (int k = 0; k < kChunks; ++k) tma_load_2d_pair(sb + k * kKvChunkBytes, &tm_kv, 64 * k, y, kb);
+        MLA_TRACE_EV(w, rank, EV_LOAD, i);
+        ld.next(p);
         return true;
       };
       auto reload_step = [&](int i) -> bool {
         const int st = i % kStages;
-        if (!mbar_wait(bar(B_QK_DONE + st), (i / kStages) & 1)) return false;
-        int b = 0, page = 0;
-        bool first = false;
-        step_info(i, b, page, first);
-        const int32_t blk = block_of(b, page);
+        if (!mbar_wait<false>(bar(B_QK_DONE + st), (i / kStages) & 1)) return false;
         const uint32_t vb = leader_bar(B_V_FULL + st);
-        mbar_arrive_expect_tx_cluster(vb, 4 * kKvChunkBytes);
+        expect_leader(B_V_FULL + st, 4 * kKvChunkBytes);
         // CTA c takes latent chunk 2q + c for the other 32 tokens of the page
         // into slot 2q + 1 - c (a chunk this CTA's PV never reads).
-        const int y = blk * 64 + 32 * (1 - (int)rank);
+        const int y = stage_blk[st] * 64 + 32 * (1 - (int)rank);
         const uint32_t sb = base + L::kv + st * kStageBytes;
         for (int q = 0; q < 4; ++q)
           tma_load_2d_pair(sb + (2 * q + 1 - rank) * kKvChunkBytes, &tm_kv, 64 * (2 * q + (int)rank), y, vb);
+        MLA_TRACE_EV(w, rank, EV_RELOAD, i);
         return true;
       };
       bool ok = true;
-      for (int i = 0; i < nsteps && i < 2 && ok; ++i) ok = load_step(i);
+      for (int i = 0; i < nsteps && i < 2 && ok; ++i) ok = load_step(i, block_of(ld));
       for (int i = 0; i < nsteps && ok; ++i) {
+        const int32_t next_blk = (i + 2 < nsteps) ? block_of(ld) : 0;  // fetched before the waits
         ok = reload_step(i);
         if (ok && i + 2 < nsteps) {
           // stage of step i+2 was used by step i-1: wait for its PV
           if (i >= 1) {
             const int j = i - 1;
-            ok = mbar_wait(bar(B_STAGE_FREE + j % kStages), (j / kStages) & 1);
+            ok = mbar_wait<false>(bar(B_STAGE_FREE + j % kStages), (j / kStages) & 1);
           }
-          if (ok) ok = load_step(i + 2);
+          if (ok) ok = load_step(i + 2, next_blk);
         }
       }
       if (!ok) fail(MLA_ERR_DEVICE_TIMEOUT);
@@ -252,6 +292,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (rank == 0 && lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
+      // descriptors of chunk 0 / k-step 0; the 14-bit start-address field
+      // (address >> 4) advances by adding the byte offset >> 4
+      const uint64_t q_desc0 = smem_desc_sw128(base + L::q, 16, 1024);
+      const uint64_t kv_desc0 = smem_desc_sw128(base + L::kv, 16, 1024);
+      const uint64_t p_desc0 = smem_desc_sw128(base + L::p, 16, 1024);
+      const uint64_t v_desc0 = smem_desc_sw128(base + L::kv, 8192, 1024);
       bool ok = true;
       int i = 0;
       int prev_seg = -1;
@@ -265,18 +311,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!mbar_wait(bar(B_P_FULL + (j & 1)), (j >> 1) & 1)) return false;
         if (!mbar_wait(bar(B_V_FULL + j % kStages), (j / kStages) & 1)) return false;
         if (first_of_seg && segidx > 0 && !mbar_wait(bar(B_O_FREE), (segidx - 1) & 1)) return false;
+        MLA_TRACE_EV(w, 0, EV_PV_READY, j);
         tc_fence_after();
-        const uint32_t sb = base + L::kv + (j % kStages) * kStageBytes;
+        const uint64_t vd = v_desc0 + (uint64_t)(((j % kStages) * kStageBytes) >> 4);
+#pragma unroll
         for (int nb = 0; nb < 2; ++nb) {
           const int shard = S == 2 ? nb : 0;
-          const uint32_t pa = base + L::p + ((j & 1) * S + shard) * kPBytes;
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = smem_desc_sw128(pa + 32 * ks, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(sb + 16384 * nb + 2048 * ks, 8192, 1024);
-            mma_f16<2>(tbase + kTmemO + 128 * nb, ad, bd, idesc_pv,
+          const uint64_t pd = p_desc0 + (uint64_t)((((j & 1) * S + shard) * kPBytes) >> 4);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16<2>(tbase + kTmemO + 128 * nb, pd + (uint64_t)(2 * ks),
+                       vd + (uint64_t)(1024 * nb + 128 * ks), idesc_pv,
                        (first_of_seg && ks == 0) ? 0u : 1u);
-          }
         }
+        MLA_TRACE_EV(w, 0, EV_PV, j);
         commit_both(B_STAGE_FREE + j % kStages);
         commit_both(B_PV_DONE + (j & 1));
         return true;
@@ -288,17 +336,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (ok) ok = mbar_wait(bar(B_KV_FULL + i % kStages), (i / kStages) & 1);
           if (ok && i >= 2) ok = mbar_wait(bar(B_S_FREE + (i & 1)), ((i >> 1) - 1) & 1);
           if (!ok) break;
+          MLA_TRACE_EV(w, 0, EV_QK, i);
           tc_fence_after();
-          const uint32_t sb = base + L::kv + (i % kStages) * kStageBytes;
+          const uint64_t bd0 = kv_desc0 + (uint64_t)(((i % kStages) * kStageBytes) >> 4);
+#pragma unroll
           for (int shard = 0; shard < S; ++shard) {
             const uint32_t d = tbase + 64 * (i & 1) + 32 * shard;
-            int n = 0;
+#pragma unroll
             for (int kc = 0; kc < kChunks; ++kc) {
               if (S == 2 && kc < 8 && (kc / 4) != shard) continue;
-              for (int ks = 0; ks < 4; ++ks, ++n) {
-                const uint64_t ad = smem_desc_sw128(base + L::q + kc * kQChunkBytes + 32 * ks, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(sb + kc * kKvChunkBytes + 32 * ks, 16, 1024);
-                mma_f16<2>(d, ad, bd, idesc_qk, n > 0 ? 1u : 0u);
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                const bool first_k = (S == 2) ? (kc == 4 * shard && ks == 0) : (kc == 0 && ks == 0);
+                mma_f16<2>(d, q_desc0 + (uint64_t)(kc * (kQChunkBytes >> 4) + 2 * ks),
+                           bd0 + (uint64_t)(kc * (kKvChunkBytes >> 4) + 2 * ks), idesc_qk,
+                           first_k ? 0u : 1u);
               }
             }
           }
@@ -337,7 +389,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto named_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
     auto wait = [&](int b, uint32_t parity) {
       if (ok && *abort_flag) ok = false;
-      if (ok) ok = mbar_wait(bar(b), parity);
+      if (ok) ok = mbar_wait<false>(bar(b), parity);
       ok = __all_sync(0xffffffffu, ok);
     };
     for_each_segment(p, w, [&](int, int b, int pb, int pe) {
@@ -349,6 +401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int sbuf = i & 1;
         uint32_t sr[S][32];
         wait(B_S_FULL + sbuf, (i >> 1) & 1);
+        if (lq == 0) MLA_TRACE_EV(w, rank, EV_S_READY, i);
         if (ok) {
           tc_fence_after();
 #pragma unroll
@@ -362,12 +415,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j) sr[s][j] = 0u;
         }
         __syncwarp();
-        if (ok && lane == 0) mbar_arrive_cluster(leader_bar(B_S_FREE + sbuf));
-        // validity of this thread's 32 tokens [tok0, tok0 + 32)
-        const int32_t blk = p.block_table[(int64_t)b * p.bt_stride + page];
-        const bool blk_ok = blk >= 0 && blk < p.num_blocks;
+        if (ok && lane == 0) arrive_leader(B_S_FREE + sbuf);
+        // visible part of this thread's 32 tokens [tok0, tok0 + 32)
         const int64_t tok0 = (int64_t)page * 64 + 32 * half;
-        const int64_t lim = (row_real && blk_ok) ? L - p.Lq + t_row : -1;  // last visible key
+        const int64_t lim = row_real ? L - p.Lq + t_row : -1;  // last visible key
         int64_t nv = lim - tok0 + 1;
         nv = nv < 0 ? 0 : (nv > 32 ? 32 : nv);
         const int nvis = (int)nv;
@@ -407,6 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         // the P buffer (i & 1) was last read by PV(i - 2)
         if (i >= 2) wait(B_PV_DONE + sbuf, ((i >> 1) - 1) & 1);
+        if (lq == 0) MLA_TRACE_EV(w, rank, EV_PBUF_FREE, i);
         if (__any_sync(0xffffffffu, rescale) && page > pb) {
           // O holds PV(i - 1) of this segment: wait for it, then scale in place
           const int j = i - 1;
@@ -449,7 +501,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_before();
         }
         __syncwarp();
-        if (ok && lane == 0) mbar_arrive_cluster(leader_bar(B_P_FULL + sbuf));
+        if (ok && lane == 0) arrive_leader(B_P_FULL + sbuf);
+        if (lq == 0) MLA_TRACE_EV(w, rank, EV_P_DONE, i);
       }
       // ---- segment epilogue: O / l and log2-sum-exp of this segment
       const int j = i - 1;
@@ -490,7 +543,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       named_sync();  // xl and the O reads of all four warps are done
       __syncwarp();
-      if (ok && lane == 0) mbar_arrive_cluster(leader_bar(B_O_FREE));
+      if (ok && lane == 0) arrive_leader(B_O_FREE);
       return true;
     });
     if (!ok) fail(MLA_ERR_DEVICE_TIMEOUT);
