@@ -158,6 +158,38 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan,
                                void* out, void* workspace, size_t workspace_bytes,
                                void* stream, const mla_run_options_t* opts);
 
+/* Decode step without a caller workspace, for callers that cannot allocate
+ * device memory where they run decode steps (an engine whose memory pool owns
+ * the whole device and forbids side allocations, or a latency-critical loop
+ * that cannot afford the implicit device synchronisation of cudaMalloc and
+ * cudaFree). The source pages have no counterpart to this entry point; it is a
+ * deployment convenience of this library.
+ *
+ * Arguments are those of mla_decode_run minus the workspace: the caller still
+ * passes every input and the output. The scratch the step needs comes from a
+ * fixed 32 MiB array in this library's device image (every GPU that loads the
+ * library holds it until the process exits). Plans whose workspace_bytes
+ * exceed 32 MiB are rejected with MLA_ERR_WORKSPACE_TOO_SMALL before any device
+ * work; the DeepSeek-V3-shaped batch of 32 x 32K tokens on 148 SMs fits.
+ * No cudaMalloc, cudaFree or other allocating call is made.
+ *
+ * The first call on a device sets up that device: it resolves the array's
+ * device address and clears its header (a synchronous memset followed by a
+ * device synchronisation). Make that first call before any stream capture.
+ * All calls in the process share the one array per device and it keeps the
+ * last call's contents; two calls whose work overlaps on the GPU (different
+ * streams, or different threads) race on it and must be serialised by the
+ * caller. Errors detected on the device are recorded in the array's status
+ * word, which this entry point does not report; use mla_decode_run with a
+ * workspace and mla_decode_read_status to diagnose them. */
+mla_status_t mla_decode_run_no_alloc(mla_plan_t plan,
+                                     const void* q_nope, const void* q_rope,
+                                     const void* kv_cache, int64_t num_blocks,
+                                     const int32_t* block_table, int32_t block_table_stride,
+                                     const int32_t* seq_lens_dev,
+                                     const void* w_uk, const void* w_uv,
+                                     void* out, void* stream);
+
 /* Clears the workspace header (status word) with an async memset on `stream`.
  * Call once after allocating a workspace, before its first run. */
 mla_status_t mla_workspace_init(void* workspace, size_t workspace_bytes, void* stream);

@@ -42,7 +42,7 @@ MLA_KERNEL_TCGEN05 = 2
 # symbols declared in include/mla_decode.h
 EXPORTED = (
     "mla_decode_plan", "mla_decode_plan_ex", "mla_decode_run", "mla_decode_run_ex",
-    "mla_workspace_init",
+    "mla_decode_run_no_alloc", "mla_workspace_init",
     "mla_decode_read_status", "mla_plan_get_info", "mla_plan_segments", "mla_plan_destroy",
     "mla_status_string", "mla_abi_version",
 )
@@ -92,6 +92,9 @@ _lib.mla_decode_run.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _
 _lib.mla_decode_run_ex.restype = ctypes.c_int
 _lib.mla_decode_run_ex.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
                                    _sz, _vp, ctypes.POINTER(mla_run_options_t)]
+_lib.mla_decode_run_no_alloc.restype = ctypes.c_int
+_lib.mla_decode_run_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp,
+                                         _vp]
 _lib.mla_workspace_init.restype = ctypes.c_int
 _lib.mla_workspace_init.argtypes = [_vp, _sz, _vp]
 _lib.mla_decode_read_status.restype = ctypes.c_int
@@ -170,6 +173,15 @@ def mla_decode_run_ex(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,
                                   block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace,
                                   workspace_bytes, stream, ctypes.byref(opts)),
            "mla_decode_run_ex")
+
+
+def mla_decode_run_no_alloc(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,
+                            block_table_stride, seq_lens_dev, w_uk, w_uv, out, stream=0) -> None:
+    """mla_decode_run without a workspace (for callers that cannot allocate
+    device memory); the scratch is a fixed 32 MiB array inside the library."""
+    _check(_lib.mla_decode_run_no_alloc(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,
+                                        block_table_stride, seq_lens_dev, w_uk, w_uv, out,
+                                        stream), "mla_decode_run_no_alloc")
 
 
 def mla_workspace_init(workspace, workspace_bytes, stream=0) -> None:

@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmla_decode.so")
-SOURCES = ["mla_decode_api.cu"]
+SOURCES = ["mla_decode_api.cu", "no_alloc.cu"]
 GENCODE = "-gencode=arch=compute_100a,code=sm_100a"
 
 
