@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "simt_kernels.cuh"
 #include "tc_decode.cuh"
+#include "tc_head_gemm.cuh"
 
 using namespace mla;
 
@@ -229,10 +230,15 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* 
 
   const bool bf16 = d.dtype == MLA_BF16;
   const int nbt = p.B * p.Lq;
-  const dim3 ga(p.H, (p.r + 127) / 128, (nbt + kAbsorbRows - 1) / kAbsorbRows);
-  if (bf16) absorb_simt_kernel<__nv_bfloat16><<<ga, 128, 0, stream>>>(p);
-  else absorb_simt_kernel<float><<<ga, 128, 0, stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  const bool tc = plan->kernel == MLA_KERNEL_TCGEN05;
+  if (tc) {
+    if (launch_absorb_tc(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
+  } else {
+    const dim3 ga(p.H, (p.r + 127) / 128, (nbt + kAbsorbRows - 1) / kAbsorbRows);
+    if (bf16) absorb_simt_kernel<__nv_bfloat16><<<ga, 128, 0, stream>>>(p);
+    else absorb_simt_kernel<float><<<ga, 128, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  }
 
   cudaEvent_t ev_start = opts ? static_cast<cudaEvent_t>(opts->decode_start_event) : nullptr;
   cudaEvent_t ev_stop = opts ? static_cast<cudaEvent_t>(opts->decode_stop_event) : nullptr;
@@ -256,13 +262,17 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* 
   }
   if (ev_stop && cudaEventRecord(ev_stop, stream) != cudaSuccess) return MLA_ERR_CUDA;
 
-  const size_t csmem = simt_combine_smem_bytes(p.r);
-  const dim3 gc(p.H, (nbt + kCombineRows - 1) / kCombineRows);
-  if (bf16 && p.S == 1) combine_simt_kernel<__nv_bfloat16, 1><<<gc, kSimtThreads, csmem, stream>>>(p);
-  else if (bf16) combine_simt_kernel<__nv_bfloat16, 2><<<gc, kSimtThreads, csmem, stream>>>(p);
-  else if (p.S == 1) combine_simt_kernel<float, 1><<<gc, kSimtThreads, csmem, stream>>>(p);
-  else combine_simt_kernel<float, 2><<<gc, kSimtThreads, csmem, stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  if (tc) {
+    if (launch_uproj_tc(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
+  } else {
+    const size_t csmem = simt_combine_smem_bytes(p.r);
+    const dim3 gc(p.H, (nbt + kCombineRows - 1) / kCombineRows);
+    if (bf16 && p.S == 1) combine_simt_kernel<__nv_bfloat16, 1><<<gc, kSimtThreads, csmem, stream>>>(p);
+    else if (bf16) combine_simt_kernel<__nv_bfloat16, 2><<<gc, kSimtThreads, csmem, stream>>>(p);
+    else if (p.S == 1) combine_simt_kernel<float, 1><<<gc, kSimtThreads, csmem, stream>>>(p);
+    else combine_simt_kernel<float, 2><<<gc, kSimtThreads, csmem, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  }
   return MLA_OK;
 }
 
@@ -290,6 +300,11 @@ int mla_debug_trace_read(unsigned long long* host, size_t n) {
   const size_t cap = sizeof(tc::g_trace) / sizeof(unsigned long long);
   if (n > cap) n = cap;
   return cudaMemcpyFromSymbol(host, tc::g_trace, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 1;
+}
+int mla_debug_trace_chunks_read(unsigned long long* host, size_t n) {
+  const size_t cap = sizeof(tc::g_trace_chunk) / sizeof(unsigned long long);
+  if (n > cap) n = cap;
+  return cudaMemcpyFromSymbol(host, tc::g_trace_chunk, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 1;
 }
 #endif
 

@@ -63,10 +63,16 @@ constexpr float kRescaleThreshold = 8.0f;    // log2 units
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;
 
+#ifndef MLA_QK_SLOTS
+#define MLA_QK_SLOTS 4
+#endif
+#ifndef MLA_V_SLOTS
+#define MLA_V_SLOTS 3
+#endif
 template <int S>
 struct Cfg {
-  static constexpr int kQkSlots = S == 1 ? 4 : 3;
-  static constexpr int kVSlots = S == 1 ? 3 : 2;
+  static constexpr int kQkSlots = S == 1 ? MLA_QK_SLOTS : 3;
+  static constexpr int kVSlots = S == 1 ? MLA_V_SLOTS : 2;
   static constexpr int kSBufs = S == 1 ? 2 : 1;   // S tiles in tensor memory (128 columns each per shard)
 };
 
@@ -78,8 +84,9 @@ struct Smem {
   static constexpr uint32_t p = v + Cfg<S>::kVSlots * kSlotBytes;
   static constexpr uint32_t xch = p + S * kPBytes;  // float [S][128] max + [S][128] l
   static constexpr uint32_t bars = xch + 2 * S * 128 * 4;
-  static constexpr uint32_t nbars = 32;
+  static constexpr uint32_t nbars = 40;
   static constexpr uint32_t misc = bars + nbars * 8;  // tmem slot, abort flag
+  static_assert(Cfg<S>::kQkSlots <= 6 && Cfg<S>::kVSlots <= 6, "barrier arrays hold 6 slots");
   static constexpr uint32_t total = misc + 64;
   static constexpr uint32_t alloc = total + 1024;     // alignment slack
 };
@@ -87,18 +94,18 @@ struct Smem {
 // barrier indices (leader = only the leader CTA's copy is used)
 enum : int {
   B_Q_FULL = 0,       // leader, count 2 (+tx)
-  B_QK_FULL = 1,      // [4] leader, count 2 (+tx)
-  B_V_FULL = 5,       // [3] leader, count 2 (+tx)
-  B_S_FREE = 8,       // [2] leader, count 8 (4 softmax warps x 2 CTAs)
-  B_P_FULL = 10,      // leader, count 8
-  B_O_FREE = 11,      // leader, count 8
-  B_QK_FREE = 12,     // [4] both, count 1 (MMA commit)
-  B_V_FREE = 16,      // [3] both, count 1
-  B_S_FULL = 19,      // [2] both, count 1
-  B_PV_DONE = 21,     // both, count 1
-  B_FINAL_QK = 22,    // leader, count 1
-  B_FINAL_PV = 23,    // leader, count 1
-  B_COUNT = 24
+  B_QK_FULL = 1,      // [6] leader, count 2 (+tx)
+  B_V_FULL = 7,       // [6] leader, count 2 (+tx)
+  B_S_FREE = 13,      // [2] leader, count 8 (4 softmax warps x 2 CTAs)
+  B_P_FULL = 15,      // leader, count 8
+  B_O_FREE = 16,      // leader, count 8
+  B_QK_FREE = 17,     // [6] both, count 1 (MMA commit)
+  B_V_FREE = 23,      // [6] both, count 1
+  B_S_FULL = 29,      // [2] both, count 1
+  B_PV_DONE = 31,     // both, count 1
+  B_FINAL_QK = 32,    // leader, count 1
+  B_FINAL_PV = 33,    // leader, count 1
+  B_COUNT = 34
 };
 
 // Optional event trace (compile with -DMLA_TRACE): SM clock of per-group events
@@ -114,8 +121,20 @@ __device__ unsigned long long g_trace[kTraceWorkers * 2 * kTraceKinds * kTraceSt
       g_trace[(((w) * 2 + (rank)) * kTraceKinds + (kind)) * kTraceSteps + (step)] = t_;   \
     }                                                                                    \
   } while (0)
+// chunk-level events of worker 0's leader CTA: QK issue / full, V issue / full
+constexpr int kTraceChunks = 1024;
+__device__ unsigned long long g_trace_chunk[4 * kTraceChunks];
+#define MLA_TRACE_CHUNK(w, rank, kind, idx)                                              \
+  do {                                                                                   \
+    if ((w) == 0 && (rank) == 0 && (idx) < (uint32_t)kTraceChunks) {                     \
+      unsigned long long t_;                                                             \
+      asm volatile("mov.u64 %0, %%clock64;" : "=l"(t_));                                 \
+      g_trace_chunk[(kind) * kTraceChunks + (idx)] = t_;                                 \
+    }                                                                                    \
+  } while (0)
 #else
 #define MLA_TRACE_EV(w, rank, kind, step) do {} while (0)
+#define MLA_TRACE_CHUNK(w, rank, kind, idx) do {} while (0)
 #endif
 enum { EV_QK_START = 0, EV_QK_END, EV_PV_START, EV_PV_END, EV_S_READY, EV_P_DONE, EV_PBUF_FREE, EV_LOAD };
 
@@ -205,8 +224,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t counts[B_COUNT];
     for (int i = 0; i < B_COUNT; ++i) counts[i] = 1;
     counts[B_Q_FULL] = 2;
-    for (int i = 0; i < 4; ++i) counts[B_QK_FULL + i] = 2;
-    for (int i = 0; i < 3; ++i) counts[B_V_FULL + i] = 2;
+    for (int i = 0; i < 6; ++i) counts[B_QK_FULL + i] = 2;
+    for (int i = 0; i < 6; ++i) counts[B_V_FULL + i] = 2;
     counts[B_S_FREE] = counts[B_S_FREE + 1] = 8;
     counts[B_P_FULL] = 8;
     counts[B_O_FREE] = 8;
@@ -276,6 +295,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t dst = base + L::qk + slot * kSlotBytes;
           tma_load_2d_pair(dst, &tm_kv, 64 * kc, y0, leader_bar(B_QK_FULL + slot));
           tma_load_2d_pair(dst + kSlotBytes / 2, &tm_kv, 64 * kc, y1, leader_bar(B_QK_FULL + slot));
+          MLA_TRACE_CHUNK(w, rank, 0, cc);
         }
         if (ok) have = g.next(p);
       }
@@ -304,6 +324,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tma_load_2d_pair(dst, &tm_kv, 64 * chunk, rows[q], leader_bar(B_V_FULL + slot));
             tma_load_2d_pair(dst + kSlotBytes / 2, &tm_kv, 64 * (chunk + 1), rows[q],
                              leader_bar(B_V_FULL + slot));
+            MLA_TRACE_CHUNK(w, rank, 2, vc);
           }
         }
         if (ok) have = g.next(p);
@@ -334,6 +355,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int slot = cc % C::kQkSlots;
           ok = mbar_wait(bar(B_QK_FULL + slot), (cc / C::kQkSlots) & 1);
           if (!ok) break;
+          MLA_TRACE_CHUNK(w, 0, 1, cc);
           tc_fence_after();
           const uint64_t ad = q_desc0 + (uint64_t)(kc * (kQChunkBytes >> 4));
           const uint64_t bd = qk_desc0 + (uint64_t)((slot * kSlotBytes) >> 4);
@@ -379,6 +401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int slot = vc % C::kVSlots;
             ok = mbar_wait(bar(B_V_FULL + slot), (vc / C::kVSlots) & 1);
             if (!ok) break;
+            MLA_TRACE_CHUNK(w, 0, 3, vc);
             tc_fence_after();
             const uint64_t pd = p_desc0 + (uint64_t)((shard * kPBytes + q * kPChunkBytes) >> 4);
             const uint64_t vd = v_desc0 + (uint64_t)((slot * kSlotBytes) >> 4);
