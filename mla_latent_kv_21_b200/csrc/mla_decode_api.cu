@@ -301,6 +301,11 @@ int mla_debug_trace_read(unsigned long long* host, size_t n) {
   if (n > cap) n = cap;
   return cudaMemcpyFromSymbol(host, tc::g_trace, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 1;
 }
+int mla_debug_trace_ns_read(unsigned long long* host, size_t n) {
+  const size_t cap = sizeof(tc::g_trace_ns) / sizeof(unsigned long long);
+  if (n > cap) n = cap;
+  return cudaMemcpyFromSymbol(host, tc::g_trace_ns, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 1;
+}
 int mla_debug_trace_chunks_read(unsigned long long* host, size_t n) {
   const size_t cap = sizeof(tc::g_trace_chunk) / sizeof(unsigned long long);
   if (n > cap) n = cap;

@@ -65,13 +65,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_local(uint32_t bar, uint32
 }
 
 // Arrive on a barrier anywhere in the cluster (bar = shared::cluster address).
+// The release is CTA-scoped on purpose: what it publishes is this CTA's own
+// shared or tensor memory, which the peer reads through the pair's tensor core,
+// not through its threads. On B200 a cluster-scoped release stalls the issuing
+// thread for ~2000 cycles while this SM has TMA loads in flight (measured: it
+// caps a 2-CTA TMA stream at ~7 B/clk per SM instead of ~20).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];"
                :: "r"(bar) : "memory");
 }
 
+// Remote expect_tx: it only carries a byte count, so no ordering is needed.
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;"
                :: "r"(bar), "r"(bytes) : "memory");
 }
 
@@ -98,8 +104,10 @@ __device__ __forceinline__ bool mbar_try_wait_cta(uint32_t bar, uint32_t parity)
 }
 
 // Bounded wait for the phase with the given parity to complete. kCluster
-// selects cluster-scope acquire (arrivals from the peer CTA's threads).
-template <bool kCluster = true>
+// selects a cluster-scope acquire; the kernels use the CTA-scope form (the
+// cluster-scope one costs throughput next to in-flight TMA loads, and the
+// peer's arrivals publish nothing that this CTA's threads read).
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   auto probe = [&]() { return kCluster ? mbar_try_wait(bar, parity) : mbar_try_wait_cta(bar, parity); };
   if (probe()) return true;
@@ -129,6 +137,16 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ math -----
+// 2^x with the SFU's approximate exp2 (PTX ex2.approx.ftz.f32: relative error
+// around 2^-22, subnormal results flushed to zero). Used where the result is
+// rounded to bf16 right away.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ---------------------------------------------------------------- tcgen05 ----

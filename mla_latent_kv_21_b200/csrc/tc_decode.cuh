@@ -82,8 +82,9 @@ struct Smem {
   static constexpr uint32_t qk = q + kQBytes;
   static constexpr uint32_t v = qk + Cfg<S>::kQkSlots * kSlotBytes;
   static constexpr uint32_t p = v + Cfg<S>::kVSlots * kSlotBytes;
-  static constexpr uint32_t xch = p + S * kPBytes;  // float [S][128] max + [S][128] l
-  static constexpr uint32_t bars = xch + 2 * S * 128 * 4;
+  // float [2][S][128] row max (double-buffered by group parity) + [S][128] l
+  static constexpr uint32_t xch = p + S * kPBytes;
+  static constexpr uint32_t bars = xch + 3 * S * 128 * 4;
   static constexpr uint32_t nbars = 40;
   static constexpr uint32_t misc = bars + nbars * 8;  // tmem slot, abort flag
   static_assert(Cfg<S>::kQkSlots <= 6 && Cfg<S>::kVSlots <= 6, "barrier arrays hold 6 slots");
@@ -105,20 +106,25 @@ enum : int {
   B_PV_DONE = 31,     // both, count 1
   B_FINAL_QK = 32,    // leader, count 1
   B_FINAL_PV = 33,    // leader, count 1
-  B_COUNT = 34
+  B_P_FREE_LO = 34,   // both, count 1: PV is done with P chunks 0, 1 (group pages 0, 1)
+  B_P_FREE_HI = 35,   // both, count 1: PV is done with P chunks 2, 3
+  B_COUNT = 36
 };
 
 // Optional event trace (compile with -DMLA_TRACE): SM clock of per-group events
 // of the first kTraceWorkers workers, read back with mla_debug_trace_read().
 #ifdef MLA_TRACE
-constexpr int kTraceWorkers = 4, kTraceKinds = 8, kTraceSteps = 64;
+constexpr int kTraceWorkers = 4, kTraceKinds = 15, kTraceSteps = 64;
 __device__ unsigned long long g_trace[kTraceWorkers * 2 * kTraceKinds * kTraceSteps];
+__device__ unsigned long long g_trace_ns[kTraceWorkers * 2 * kTraceKinds * kTraceSteps];
 #define MLA_TRACE_EV(w, rank, kind, step)                                                \
   do {                                                                                   \
     if ((w) < kTraceWorkers && (step) < kTraceSteps) {                                   \
-      unsigned long long t_;                                                             \
+      unsigned long long t_, n_;                                                         \
       asm volatile("mov.u64 %0, %%clock64;" : "=l"(t_));                                 \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(n_));                             \
       g_trace[(((w) * 2 + (rank)) * kTraceKinds + (kind)) * kTraceSteps + (step)] = t_;   \
+      g_trace_ns[(((w) * 2 + (rank)) * kTraceKinds + (kind)) * kTraceSteps + (step)] = n_;\
     }                                                                                    \
   } while (0)
 // chunk-level events of worker 0's leader CTA: QK issue / full, V issue / full
@@ -136,7 +142,8 @@ __device__ unsigned long long g_trace_chunk[4 * kTraceChunks];
 #define MLA_TRACE_EV(w, rank, kind, step) do {} while (0)
 #define MLA_TRACE_CHUNK(w, rank, kind, idx) do {} while (0)
 #endif
-enum { EV_QK_START = 0, EV_QK_END, EV_PV_START, EV_PV_END, EV_S_READY, EV_P_DONE, EV_PBUF_FREE, EV_LOAD };
+enum { EV_QK_START = 0, EV_QK_END, EV_PV_START, EV_PV_END, EV_S_READY, EV_P_DONE, EV_PBUF_FREE, EV_LOAD,
+       EV_PASS1, EV_PASS2, EV_SYNC1, EV_LD0 };
 
 // Sequential walk over a worker's page groups: sequence b, first page and
 // page count of the group (1..4), first-group-of-segment flag, segment index.
@@ -275,7 +282,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // QK of the previous group (the previous segment's last) must be
             // done with Q before it is overwritten
             const int j = gi - 1;
-            ok = mbar_wait<false>(bar(B_S_FULL + j % C::kSBufs), (j / C::kSBufs) & 1);
+            ok = mbar_wait(bar(B_S_FULL + j % C::kSBufs), (j / C::kSBufs) & 1);
             if (!ok) break;
           }
           expect_leader(B_Q_FULL, kQBytes);
@@ -289,7 +296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kc = 0; kc < kChunks && ok; ++kc, ++cc) {
           const int slot = cc % C::kQkSlots;
           if (cc >= (uint32_t)C::kQkSlots)
-            ok = mbar_wait<false>(bar(B_QK_FREE + slot), ((cc / C::kQkSlots) - 1) & 1);
+            ok = mbar_wait(bar(B_QK_FREE + slot), ((cc / C::kQkSlots) - 1) & 1);
           if (!ok) break;
           expect_leader(B_QK_FULL + slot, kSlotBytes);
           const uint32_t dst = base + L::qk + slot * kSlotBytes;
@@ -312,11 +319,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       while (have && ok) {
         int rows[kGroupPages];
         for (int q = 0; q < kGroupPages; ++q) rows[q] = page_row(g.b, g.page + q, q < g.npages);
-        for (int nb = 0; nb < 2 && ok; ++nb) {
-          for (int q = 0; q < kGroupPages && ok; ++q, ++vc) {
+        for (int q = 0; q < kGroupPages && ok; ++q) {
+          for (int nb = 0; nb < 2 && ok; ++nb, ++vc) {
             const int slot = vc % C::kVSlots;
             if (vc >= (uint32_t)C::kVSlots)
-              ok = mbar_wait<false>(bar(B_V_FREE + slot), ((vc / C::kVSlots) - 1) & 1);
+              ok = mbar_wait(bar(B_V_FREE + slot), ((vc / C::kVSlots) - 1) & 1);
             if (!ok) break;
             expect_leader(B_V_FULL + slot, kSlotBytes);
             const uint32_t dst = base + L::v + slot * kSlotBytes;
@@ -376,7 +383,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         have = g.next(p);
       }
       tc_commit<2>(bar(B_FINAL_QK));
-      if (!mbar_wait<false>(bar(B_FINAL_QK), 0)) ok = false;
+      if (!mbar_wait(bar(B_FINAL_QK), 0)) ok = false;
       if (!ok) fail(MLA_ERR_DEVICE_TIMEOUT);
     }
     __syncwarp();
@@ -395,9 +402,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (ok && g.first && g.seg > 0) ok = mbar_wait(bar(B_O_FREE), (g.seg - 1) & 1);
         if (!ok) break;
         MLA_TRACE_EV(w, 0, EV_PV_START, gi);
-        for (int nb = 0; nb < 2 && ok; ++nb) {
-          const int shard = S == 2 ? nb : 0;
-          for (int q = 0; q < kGroupPages && ok; ++q, ++vc) {
+        // page-major: P chunks 0, 1 are released half way through
+        for (int q = 0; q < kGroupPages && ok; ++q) {
+          for (int nb = 0; nb < 2 && ok; ++nb, ++vc) {
+            const int shard = S == 2 ? nb : 0;
             const int slot = vc % C::kVSlots;
             ok = mbar_wait(bar(B_V_FULL + slot), (vc / C::kVSlots) & 1);
             if (!ok) break;
@@ -412,14 +420,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                          (g.first && q == 0 && ks == 0) ? 0u : 1u);
             commit_both(B_V_FREE + slot);
           }
+          if (q == 1) commit_both(B_P_FREE_LO);
         }
         if (!ok) break;
         MLA_TRACE_EV(w, 0, EV_PV_END, gi);
+        commit_both(B_P_FREE_HI);
         commit_both(B_PV_DONE);
         have = g.next(p);
       }
       tc_commit<2>(bar(B_FINAL_PV));
-      if (!mbar_wait<false>(bar(B_FINAL_PV), 0)) ok = false;
+      if (!mbar_wait(bar(B_FINAL_PV), 0)) ok = false;
       if (!ok) fail(MLA_ERR_DEVICE_TIMEOUT);
     }
     __syncwarp();
@@ -436,12 +446,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int t_row = row_real ? row / p.H : 0;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     bool ok = true;
-    float* xmax = xch;                             // [S][128]
-    float* xl = xch + S * 128;                     // [S][128]
+    float* xl = xch + 2 * S * 128;                 // [S][128]
     auto named_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
     auto wait = [&](int b, uint32_t parity) {
       if (ok && *abort_flag) ok = false;
-      if (ok) ok = mbar_wait<false>(bar(b), parity);
+      if (ok) ok = mbar_wait(bar(b), parity);
       ok = __all_sync(0xffffffffu, ok);
     };
     GroupCursor g;
@@ -454,10 +463,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int s = 0; s < S; ++s) { m[s] = -INFINITY; l[s] = 0.f; }
       }
       const int sb = gi % C::kSBufs;
+      float* xmax = xch + (gi & 1) * S * 128;      // this group's [S][128] row maxima
       const int64_t L = p.seq_lens[g.b];
       // this thread's 128 tokens: group pages 2 half, 2 half + 1; the visible
       // ones are the first nvis (pages past the group's end or past the causal
-      // limit are masked)
+      // limit are masked); nvis is uniform across the warp
       const int64_t key0 = (int64_t)(g.page + 2 * half) * 64;
       const int64_t lim = row_real ? L - p.Lq + t_row : -1;  // last visible key
       int64_t nv = lim - key0 + 1;
@@ -469,92 +479,110 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       wait(B_S_FULL + sb, (gi / C::kSBufs) & 1);
       if (lq == 0) MLA_TRACE_EV(w, rank, EV_S_READY, gi);
       if (ok) tc_fence_after();
-      // pass 1: row max over this thread's tokens
-      float mt_own[S];
-#pragma unroll
-      for (int s = 0; s < S; ++s) {
-        float mx = -INFINITY;
-        if (ok) {
 #pragma unroll 1
-          for (int c0 = 0; c0 < 128; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(tbase + lane_off + sb * 128 * S + 128 * s + c0, r);
-            tmem_wait_ld();
+      for (int s = 0; s < S; ++s) {
+        // one pass over tensor memory: the thread's 128 scores of shard s
+        uint32_t r[128];
+        if (ok) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c0 + j < nvis) mx = fmaxf(mx, __uint_as_float(r[j]));
+          for (int c0 = 0; c0 < 128; c0 += 32)
+            tmem_ld32(tbase + lane_off + sb * 128 * S + 128 * s + c0,
+                      *reinterpret_cast<uint32_t(*)[32]>(r + c0));
+          tmem_wait_ld();
+        }
+        if (s == S - 1) {
+          // every score of this S buffer is in registers: QK may reuse it
+          if (ok) tc_fence_before();
+          __syncwarp();
+          if (ok && lane == 0) arrive_leader(B_S_FREE + sb);
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+        if (ok) {
+          if (nvis >= 128) {
+#pragma unroll
+            for (int j = 0; j < 128; j += 2) {
+              mx0 = fmaxf(mx0, __uint_as_float(r[j]));
+              mx1 = fmaxf(mx1, __uint_as_float(r[j + 1]));
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 128; ++j)
+              if (j < nvis) mx0 = fmaxf(mx0, __uint_as_float(r[j]));
           }
         }
-        mt_own[s] = mx * p.scale_log2;
-        xmax[s * 128 + lq] = mt_own[s];
-      }
-      named_sync();
-      float alpha[S];
-      bool rescale = false;
-#pragma unroll
-      for (int s = 0; s < S; ++s) {
-        const float mt = fmaxf(mt_own[s], xmax[s * 128 + (lq ^ 64)]);
+        const float mt_own = fmaxf(mx0, mx1) * p.scale_log2;
+        xmax[s * 128 + lq] = mt_own;
+        if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PASS1, gi);
+        named_sync();
+        // row max over both token halves (the other half lives in lane lq ^ 64)
+        const float mt = fmaxf(mt_own, xmax[s * 128 + (lq ^ 64)]);
         float mu = m[s];
         if (m[s] == -INFINITY || mt > m[s] + kRescaleThreshold) mu = fmaxf(mt, m[s]);
-        alpha[s] = 1.f;
-        if (mu != m[s] && m[s] != -INFINITY) {
-          alpha[s] = exp2f(m[s] - mu);
-          rescale = true;
-        }
+        float alpha = 1.f;
+        const bool rescale = mu != m[s] && m[s] != -INFINITY;
+        if (rescale) alpha = ex2_approx(m[s] - mu);
         m[s] = mu;
-      }
-      // pass 2: P = exp2(s * scale - m), packed bf16, row sums
-      uint32_t pk[S][64];
+        // P = 2^(score * scale - m) in bf16 pairs, row sum in four partial sums
+        uint32_t pk[64];
+        float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
+        if (ok && mu != -INFINITY) {
+          if (nvis >= 128) {
 #pragma unroll
-      for (int s = 0; s < S; ++s) {
-        float ps = 0.f;
-        const float mu = m[s];
-#pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t r[32];
-          if (ok) {
-            tmem_ld32(tbase + lane_off + sb * 128 * S + 128 * s + c0, r);
-            tmem_wait_ld();
-          }
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            float p0 = 0.f, p1 = 0.f;
-            if (ok && mu != -INFINITY) {
-              if (c0 + j < nvis) p0 = exp2f(fmaf(__uint_as_float(r[j]), p.scale_log2, -mu));
-              if (c0 + j + 1 < nvis) p1 = exp2f(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, -mu));
+            for (int j = 0; j < 128; j += 4) {
+              const float p0 = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, -mu));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, -mu));
+              const float p2 = ex2_approx(fmaf(__uint_as_float(r[j + 2]), p.scale_log2, -mu));
+              const float p3 = ex2_approx(fmaf(__uint_as_float(r[j + 3]), p.scale_log2, -mu));
+              ps0 += p0; ps1 += p1; ps2 += p2; ps3 += p3;
+              __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
+              __nv_bfloat162 h1 = __floats2bfloat162_rn(p2, p3);
+              pk[j >> 1] = *reinterpret_cast<uint32_t*>(&h0);
+              pk[(j >> 1) + 1] = *reinterpret_cast<uint32_t*>(&h1);
             }
-            ps += p0 + p1;
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            pk[s][(c0 + j) >> 1] = *reinterpret_cast<uint32_t*>(&h2);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 128; j += 2) {
+              float p0 = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, -mu));
+              float p1 = ex2_approx(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, -mu));
+              p0 = j < nvis ? p0 : 0.f;
+              p1 = j + 1 < nvis ? p1 : 0.f;
+              ps0 += p0; ps1 += p1;
+              __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
+              pk[j >> 1] = *reinterpret_cast<uint32_t*>(&h0);
+            }
           }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) pk[j] = 0u;
         }
-        l[s] = l[s] * alpha[s] + ps;
-      }
-      if (ok) tc_fence_before();
-      __syncwarp();
-      if (ok && lane == 0) arrive_leader(B_S_FREE + sb);
-      // P buffer and O: PV of the previous group must be complete
-      if (gi >= 1) wait(B_PV_DONE, (gi - 1) & 1);
-      if (lq == 0) MLA_TRACE_EV(w, rank, EV_PBUF_FREE, gi);
-      if (ok && !g.first && __any_sync(0xffffffffu, rescale)) {
-        tc_fence_after();
+        l[s] = l[s] * alpha + ((ps0 + ps1) + (ps2 + ps3));
+        if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PASS2, gi);
+        // this warp's P chunks (2 half, 2 half + 1): the previous group's PV
+        // must be done with them
+        if (s == 0 && gi >= 1) wait(half ? B_P_FREE_HI : B_P_FREE_LO, (gi - 1) & 1);
+        if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PBUF_FREE, gi);
+        // rescale this shard's O columns (all 256 for one shard, 128 each for
+        // two) once the previous group's PV is complete
+        if (!g.first && __any_sync(0xffffffffu, rescale)) {
+          wait(B_PV_DONE, (gi - 1) & 1);
+        }
+        if (ok && !g.first && __any_sync(0xffffffffu, rescale)) {
+          tc_fence_after();
+          constexpr int kOCols = 256 / S;
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
-          const float a = alpha[S == 2 ? (c >> 7) : 0];
-          uint32_t o[32];
-          tmem_ld32(tbase + lane_off + kTmemO + c, o);
-          tmem_wait_ld();
+          for (int c = 0; c < kOCols; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tbase + lane_off + kTmemO + kOCols * s + c, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
-          tmem_st32(tbase + lane_off + kTmemO + c, o);
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(tbase + lane_off + kTmemO + kOCols * s + c, o);
+          }
+          tmem_wait_st();
         }
-        tmem_wait_st();
-      }
-      if (ok) {
-        // P -> shared memory, K-major 128-byte swizzle: row rloc, tokens
-        // [128 half, +128) = chunks 2 half, 2 half + 1, 16-byte units 0..7 each
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
+        if (ok) {
+          // P -> shared memory, K-major 128-byte swizzle: row rloc, tokens
+          // [128 half, +128) = chunks 2 half, 2 half + 1, 16-byte units 0..7 each
           uint8_t* pbuf = gbase + L::p + s * kPBytes;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
@@ -562,10 +590,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int u = 0; u < 8; ++u)
               *reinterpret_cast<uint4*>(chunk + sw128(rloc, u)) =
-                  make_uint4(pk[s][32 * t + 4 * u], pk[s][32 * t + 4 * u + 1],
-                             pk[s][32 * t + 4 * u + 2], pk[s][32 * t + 4 * u + 3]);
+                  make_uint4(pk[32 * t + 4 * u], pk[32 * t + 4 * u + 1],
+                             pk[32 * t + 4 * u + 2], pk[32 * t + 4 * u + 3]);
           }
         }
+      }
+      if (ok) {
         fence_proxy_async_smem();
         tc_fence_before();
       }
