@@ -141,7 +141,8 @@ mla_status_t mla_plan_get_info(mla_plan_t plan, mla_plan_info_t* info) {
   info->kernel = plan->kernel;
   info->num_workers = plan->W;
   info->num_split_slots = plan->W + plan->B - 1;
-  info->launches_per_run = 3;
+  // tcgen05: absorb, decode, split merge, up-projection; SIMT: absorb, decode, combine
+  info->launches_per_run = plan->kernel == MLA_KERNEL_TCGEN05 ? 4 : 3;
   info->total_pages = plan->G;
   info->workspace_bytes = plan->layout.total;
   return MLA_OK;
@@ -263,7 +264,7 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* 
   if (ev_stop && cudaEventRecord(ev_stop, stream) != cudaSuccess) return MLA_ERR_CUDA;
 
   if (tc) {
-    if (launch_uproj_tc(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
+    if (launch_combine_tc(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
   } else {
     const size_t csmem = simt_combine_smem_bytes(p.r);
     const dim3 gc(p.H, (nbt + kCombineRows - 1) / kCombineRows);
@@ -305,6 +306,16 @@ int mla_debug_trace_ns_read(unsigned long long* host, size_t n) {
   const size_t cap = sizeof(tc::g_trace_ns) / sizeof(unsigned long long);
   if (n > cap) n = cap;
   return cudaMemcpyFromSymbol(host, tc::g_trace_ns, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 1;
+}
+int mla_debug_trace_cta_read(unsigned long long* host, size_t n) {
+  const size_t cap = sizeof(tc::g_trace_cta) / sizeof(unsigned long long);
+  if (n > cap) n = cap;
+  return cudaMemcpyFromSymbol(host, tc::g_trace_cta, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 1;
+}
+int mla_debug_trace_hg_read(unsigned long long* host, size_t n) {
+  const size_t cap = sizeof(hg::g_hg_trace) / sizeof(unsigned long long);
+  if (n > cap) n = cap;
+  return cudaMemcpyFromSymbol(host, hg::g_hg_trace, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 1;
 }
 int mla_debug_trace_chunks_read(unsigned long long* host, size_t n) {
   const size_t cap = sizeof(tc::g_trace_chunk) / sizeof(unsigned long long);

@@ -64,10 +64,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;
 
 #ifndef MLA_QK_SLOTS
-#define MLA_QK_SLOTS 4
+#define MLA_QK_SLOTS 3
 #endif
 #ifndef MLA_V_SLOTS
-#define MLA_V_SLOTS 3
+#define MLA_V_SLOTS 4
 #endif
 template <int S>
 struct Cfg {
@@ -127,6 +127,16 @@ __device__ unsigned long long g_trace_ns[kTraceWorkers * 2 * kTraceKinds * kTrac
       g_trace_ns[(((w) * 2 + (rank)) * kTraceKinds + (kind)) * kTraceSteps + (step)] = n_;\
     }                                                                                    \
   } while (0)
+// per CTA: globaltimer at entry, after setup, at the start of teardown, at exit
+__device__ unsigned long long g_trace_cta[1024 * 4];
+#define MLA_TRACE_CTA(k)                                                                  \
+  do {                                                                                   \
+    if (threadIdx.x == 0 && blockIdx.x < 1024) {                                         \
+      unsigned long long n_;                                                             \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(n_));                             \
+      g_trace_cta[blockIdx.x * 4 + (k)] = n_;                                            \
+    }                                                                                    \
+  } while (0)
 // chunk-level events of worker 0's leader CTA: QK issue / full, V issue / full
 constexpr int kTraceChunks = 1024;
 __device__ unsigned long long g_trace_chunk[4 * kTraceChunks];
@@ -141,6 +151,7 @@ __device__ unsigned long long g_trace_chunk[4 * kTraceChunks];
 #else
 #define MLA_TRACE_EV(w, rank, kind, step) do {} while (0)
 #define MLA_TRACE_CHUNK(w, rank, kind, idx) do {} while (0)
+#define MLA_TRACE_CTA(k) do {} while (0)
 #endif
 enum { EV_QK_START = 0, EV_QK_END, EV_PV_START, EV_PV_END, EV_S_READY, EV_P_DONE, EV_PBUF_FREE, EV_LOAD,
        EV_PASS1, EV_PASS2, EV_SYNC1, EV_LD0 };
@@ -201,7 +212,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   using L = Smem<S>;
   using C = Cfg<S>;
   extern __shared__ uint8_t smem_raw[];
-  if (!*p.lengths_ok) return;  // uniform across the pair
+  MLA_TRACE_CTA(0);
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -248,6 +259,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  // the setup above overlaps the previous kernel; from here on its results
+  // (the absorbed queries, the page prefix sums) are read
+  grid_launch_dependents();
+  grid_dependency_wait();
+  const bool run = *p.lengths_ok != 0;  // uniform across the pair
+  MLA_TRACE_CTA(1);
 
   auto fail = [&](int code) {
     record_error(p.status, code);
@@ -267,7 +284,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     return blk * 64;
   };
 
-  if (warp == 0) {
+  if (!run) {
+    // invalid lengths (reported by the length scan): nothing to do
+  } else if (warp == 0) {
     // --------------------------------------------- Q and QK chunk producer --
     if (lane == 0) {
       prefetch_tmap(&tm_kv);
@@ -650,10 +669,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   __syncwarp();
 
+  MLA_TRACE_CTA(2);
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
   if (warp == 1) tmem_dealloc<2>(tbase, kTmemCols);
+  MLA_TRACE_CTA(3);
 }
 
 // ------------------------------------------------------------------ host ---
@@ -698,14 +719,16 @@ inline cudaError_t launch_tc_decode(const RunParams& p, cudaStream_t stream) {
     e = cudaFuncSetAttribute(tc::decode_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tc::Smem<1>::alloc);
     if (e != cudaSuccess) return e;
-    tc::decode_tc_kernel<1><<<2 * p.W, tc::kThreads, tc::Smem<1>::alloc, stream>>>(tm_kv, tm_q, p);
+    e = launch_dependent(tc::decode_tc_kernel<1>, dim3(2 * p.W), dim3(tc::kThreads), tc::Smem<1>::alloc,
+                         stream, tm_kv, tm_q, p);
   } else {
     e = cudaFuncSetAttribute(tc::decode_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tc::Smem<2>::alloc);
     if (e != cudaSuccess) return e;
-    tc::decode_tc_kernel<2><<<2 * p.W, tc::kThreads, tc::Smem<2>::alloc, stream>>>(tm_kv, tm_q, p);
+    e = launch_dependent(tc::decode_tc_kernel<2>, dim3(2 * p.W), dim3(tc::kThreads), tc::Smem<2>::alloc,
+                         stream, tm_kv, tm_q, p);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace mla

@@ -25,21 +25,38 @@ namespace mla {
 namespace hg {
 
 constexpr int kThreads = 256;
-constexpr int kMaxN = 256;               // query rows per CTA (MMA N)
+
+#ifdef MLA_TRACE
+// per CTA (blockIdx.x < 256): globaltimer at entry, operands landed, MMA done, exit
+__device__ unsigned long long g_hg_trace[2][256 * 4];
+#define MLA_HG_TRACE(kern, k)                                                             \
+  do {                                                                                   \
+    if (blockIdx.x < 256 && blockIdx.y == 0) {                                           \
+      unsigned long long n_;                                                             \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(n_));                             \
+      g_hg_trace[kern][blockIdx.x * 4 + (k)] = n_;                                       \
+    }                                                                                    \
+  } while (0)
+#else
+#define MLA_HG_TRACE(kern, k) do {} while (0)
+#endif
 
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk16) {
   return row * 128 + ((chunk16 ^ (row & 7)) << 4);
 }
 
 // ---------------------------------------------------------------------------
-// absorb: grid (H, 4 latent tiles of 128, ceil(rows / 256)); block 256.
-// Shared memory: W tile [K = 128 d_nope][M = 128 latent] as 2 MN-major groups
-// of 64 latent columns (16 KB each); q_nope rows [N][128] as 2 K-major chunks.
+// absorb: grid (H, ceil(rows / 128)); block 256. One CTA reads all of W_UK[h]
+// (128 KB) once and computes the 4 latent tiles of 128 into 4 tensor-memory
+// accumulators, so 128 heads run as one wave.
+// Shared memory: W_UK[h] [K = 128 d_nope][512 latent] as 8 MN-major groups of
+// 64 latent columns (16 KB each); q_nope rows [N][128] as 2 K-major chunks.
 // ---------------------------------------------------------------------------
+constexpr int kAbsorbMaxN = 128;         // query rows per absorb CTA
 struct AbsorbSmem {
-  static constexpr uint32_t w = 0;                   // 32 KB
-  static constexpr uint32_t x = 32768;               // 2 x N x 128 B <= 64 KB
-  static constexpr uint32_t bars = x + 2 * kMaxN * 128;
+  static constexpr uint32_t w = 0;                             // 128 KB
+  static constexpr uint32_t x = 131072;                        // 2 x N x 128 B <= 32 KB
+  static constexpr uint32_t bars = x + 2 * kAbsorbMaxN * 128;
   static constexpr uint32_t misc = bars + 64;
   static constexpr uint32_t alloc = misc + 64 + 1024;
 };
@@ -50,66 +67,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   using namespace ptx;
   extern __shared__ uint8_t smem_raw[];
   // page prefix sums and length check of this run (all 256 threads of one block)
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) scan_lengths(p);
+  if (threadIdx.x == 0) MLA_HG_TRACE(0, 0);
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const int h = blockIdx.x, mt = blockIdx.y, nt = blockIdx.z;
+  const int h = blockIdx.x;
   const int nbt = p.B * p.Lq;
-  const int row0 = nt * kMaxN;
-  const int nrows = min(kMaxN, nbt - row0);
+  const int row0 = blockIdx.y * kAbsorbMaxN;
+  const int nrows = min(kAbsorbMaxN, nbt - row0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar_full = base + AbsorbSmem::bars, bar_done = bar_full + 8;
+  const uint32_t bar_w = base + AbsorbSmem::bars, bar_x = bar_w + 8, bar_done = bar_w + 16;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(gbase + AbsorbSmem::misc);
+  // tensor memory: 4 accumulators of n_pad columns (n_pad <= 128)
+  const uint32_t tcols = 4 * n_pad <= 32 ? 32 : 4 * n_pad <= 64 ? 64 : 4 * n_pad <= 128 ? 128 :
+                         4 * n_pad <= 256 ? 256 : 512;
   if (threadIdx.x == 0) {
-    mbar_init(bar_full, 1);
+    mbar_init(bar_w, 1);
+    mbar_init(bar_x, 1);
     mbar_init(bar_done, 1);
     fence_mbarrier_init_cluster();
+    // the weights do not depend on the previous kernel: fetch them at once
+    prefetch_tmap(&tm_wuk);
+    prefetch_tmap(&tm_qn);
+    mbar_arrive_expect_tx_local(bar_w, 8 * 16384);
+    for (int j = 0; j < 8; ++j)  // W_UK[h][:, 64 j .. +64], all 128 d rows
+      tma_load_2d(base + AbsorbSmem::w + 16384 * j, &tm_wuk, 64 * j, h * p.dn, bar_w);
   }
   __syncwarp();
   if (warp == 0) {
-    tmem_alloc<1>(base + AbsorbSmem::misc, 256);
+    tmem_alloc<1>(base + AbsorbSmem::misc, tcols);
     tmem_relinquish<1>();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  bool ok = true;
+  // q_nope may come from the previous kernel, and that kernel may still read
+  // the workspace (prefix sums, query buffer) this kernel writes
+  grid_launch_dependents();
+  grid_dependency_wait();
+  // page prefix sums and length check of this run (all 256 threads of one block)
+  if (blockIdx.x == 0 && blockIdx.y == 0) scan_lengths(p);
   if (threadIdx.x == 0) {
-    prefetch_tmap(&tm_wuk);
-    prefetch_tmap(&tm_qn);
-    const uint32_t bytes = 2 * 16384 + 2 * n_pad * 128;
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-                 :: "r"(bar_full), "r"(bytes) : "memory");
-    for (int j = 0; j < 2; ++j)  // W_UK[h][:, 128 mt + 64 j .. +64], all 128 d rows
-      asm volatile(
-          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-          :: "r"(base + AbsorbSmem::w + 16384 * j), "l"(reinterpret_cast<uint64_t>(&tm_wuk)),
-             "r"(128 * mt + 64 * j), "r"(h * p.dn), "r"(bar_full) : "memory");
+    mbar_arrive_expect_tx_local(bar_x, 2 * n_pad * 128);
     for (int kc = 0; kc < 2; ++kc)  // q_nope rows [row0, row0 + n_pad), d chunk kc
-      asm volatile(
-          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-          :: "r"(base + AbsorbSmem::x + kc * n_pad * 128), "l"(reinterpret_cast<uint64_t>(&tm_qn)),
-             "r"(h * p.dn + 64 * kc), "r"(row0), "r"(bar_full) : "memory");
-    ok = mbar_wait<false>(bar_full, 0);
-    if (ok) {
+      tma_load_2d(base + AbsorbSmem::x + kc * n_pad * 128, &tm_qn, h * p.dn + 64 * kc, row0, bar_x);
+    if (mbar_wait(bar_w, 0) && mbar_wait(bar_x, 0)) {
+      MLA_HG_TRACE(0, 1);
       tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(128, n_pad, 1, 0);
-      const uint64_t a0 = smem_desc_sw128(base + AbsorbSmem::w, 16384, 1024);
       const uint64_t b0 = smem_desc_sw128(base + AbsorbSmem::x, 16, 1024);
-      for (int ks = 0; ks < 8; ++ks) {  // K = 128 = 8 x 16
-        const uint64_t ad = a0 + (uint64_t)(128 * ks);  // 16 K rows x 128 B
-        const uint64_t bd = b0 + (uint64_t)(((ks >> 2) * n_pad * 128) >> 4) + (uint64_t)(2 * (ks & 3));
-        mma_f16<1>(tbase, ad, bd, idesc, ks > 0 ? 1u : 0u);
+      for (int mt = 0; mt < 4; ++mt) {  // latent tile [128 mt, +128): groups 2 mt, 2 mt + 1
+        const uint64_t a0 = smem_desc_sw128(base + AbsorbSmem::w + 32768 * mt, 16384, 1024);
+        for (int ks = 0; ks < 8; ++ks) {  // K = 128 = 8 x 16
+          const uint64_t ad = a0 + (uint64_t)(128 * ks);  // 16 K rows x 128 B
+          const uint64_t bd = b0 + (uint64_t)(((ks >> 2) * n_pad * 128) >> 4) + (uint64_t)(2 * (ks & 3));
+          mma_f16<1>(tbase + mt * n_pad, ad, bd, idesc, ks > 0 ? 1u : 0u);
+        }
       }
       tc_commit<1>(bar_done);
     } else {
       record_error(p.status, MLA_ERR_DEVICE_TIMEOUT);
     }
   }
-  // q_rope columns of the packed query rows (tile 0 only)
-  if (mt == 0) {
+  // q_rope columns of the packed query rows
+  {
     const __nv_bfloat16* q_rope = static_cast<const __nv_bfloat16*>(p.q_rope);
     __nv_bfloat16* q = static_cast<__nv_bfloat16*>(p.q);
     for (int idx = threadIdx.x; idx < nrows * p.dr; idx += blockDim.x) {
@@ -118,21 +140,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncwarp();
-  if (warp < 4) {
-    const bool done = mbar_wait<false>(bar_done, 0);
+  {
+    // warps w and w + 4 share lane quadrant w % 4: tiles {0, 1} and {2, 3}
+    const bool done = mbar_wait(bar_done, 0);
+    if (threadIdx.x == 0) MLA_HG_TRACE(0, 2);
     if (__all_sync(0xffffffffu, done)) {
       tc_fence_after();
       __nv_bfloat16* q = static_cast<__nv_bfloat16*>(p.q);
-      const int m = 32 * warp + lane;  // latent column within the tile
-      for (int c0 = 0; c0 < n_pad; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tbase + ((uint32_t)(32 * warp) << 16) + c0, r);
-        tmem_wait_ld();
-        for (int j = 0; j < 32; ++j) {
-          const int i = c0 + j;
-          if (i < nrows)
-            q[((int64_t)(row0 + i) * p.H + h) * (p.r + p.dr) + 128 * mt + m] =
-                __float2bfloat16_rn(__uint_as_float(r[j]));
+      const int quad = warp & 3;
+      const int m = 32 * quad + lane;  // latent column within a tile
+      for (int mt = 2 * (warp >> 2); mt < 2 * (warp >> 2) + 2; ++mt) {
+        for (int c0 = 0; c0 < n_pad; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tbase + ((uint32_t)(32 * quad) << 16) + mt * n_pad + c0, r);
+          tmem_wait_ld();
+          for (int j = 0; j < 32; ++j) {
+            const int i = c0 + j;
+            if (i < nrows)
+              q[((int64_t)(row0 + i) * p.H + h) * (p.r + p.dr) + 128 * mt + m] =
+                  __float2bfloat16_rn(__uint_as_float(r[j]));
+          }
         }
       }
     } else if (lane == 0) {
@@ -141,30 +168,107 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc<1>(tbase, 256);
+  if (warp == 0) tmem_dealloc<1>(tbase, tcols);
+  if (threadIdx.x == 0) MLA_HG_TRACE(0, 3);
 }
 
 // ---------------------------------------------------------------------------
-// combine + up-projection: grid (H, ceil(rows / 256)); block 256.
+// combine: o_lat = log-sum-exp merge of a row's split partials, per TPLA shard.
+// One thread per (query row, head, 8 latent columns); the 64 threads of a row
+// read each partial row as 2 KB of consecutive bytes. Writes bf16 o_lat
+// [B * Lq * H, r] into the absorbed-query buffer, which the decode no longer
+// needs. grid ceil(B * Lq * H * 64 / 256), block 256.
+// ---------------------------------------------------------------------------
+constexpr int kMergeThreads = 256;
+
+template <int S>
+__global__ void __launch_bounds__(kMergeThreads)
+    merge_lat_kernel(RunParams p) {
+  using namespace ptx;
+  grid_launch_dependents();
+  grid_dependency_wait();  // the partials of the decode kernel
+  if (!*p.lengths_ok) return;
+  const int units = p.r / 8;
+  const int64_t nitems = (int64_t)p.B * p.Lq * p.H * units;
+  const int64_t idx = (int64_t)blockIdx.x * kMergeThreads + threadIdx.x;
+  if (idx >= nitems) return;
+  const int unit = (int)(idx % units);
+  const int64_t rr = idx / units;                  // (b, t) * H + h
+  const int h = (int)(rr % p.H);
+  const int bt = (int)(rr / p.H);
+  const int b = bt / p.Lq, t = bt % p.Lq, row = t * p.H + h;
+  const int c0 = unit * 8, s = c0 / (p.r / S);
+  const int64_t G = p.cum[p.B];
+  const int64_t lo = page_owner(p.cum[b], G, p.W) + b;
+  const int64_t hi = page_owner(p.cum[b + 1] - 1, G, p.W) + b;
+  const float* lse = p.lse_part + (int64_t)row * S + s;
+  const int64_t lstride = (int64_t)p.rows * S;
+  const float* op = p.o_part + (int64_t)row * p.r + c0;
+  const int64_t ostride = (int64_t)p.rows * p.r;
+  float mx = -INFINITY;
+  for (int64_t slot = lo; slot <= hi; ++slot) mx = fmaxf(mx, lse[slot * lstride]);
+  float sum = 0.f, acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+  for (int64_t j0 = lo; j0 <= hi; j0 += 4) {
+    float l[4];
+    float4 v0[4], v1[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t slot = j0 + k;
+      if (slot <= hi) {
+        l[k] = lse[slot * lstride];
+        const float4* q4 = reinterpret_cast<const float4*>(op + slot * ostride);
+        v0[k] = q4[0];
+        v1[k] = q4[1];
+      } else {
+        l[k] = -INFINITY;
+        v0[k] = v1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float wk = exp2f(l[k] - mx);
+      sum += wk;
+      acc[0] = fmaf(wk, v0[k].x, acc[0]); acc[1] = fmaf(wk, v0[k].y, acc[1]);
+      acc[2] = fmaf(wk, v0[k].z, acc[2]); acc[3] = fmaf(wk, v0[k].w, acc[3]);
+      acc[4] = fmaf(wk, v1[k].x, acc[4]); acc[5] = fmaf(wk, v1[k].y, acc[5]);
+      acc[6] = fmaf(wk, v1[k].z, acc[6]); acc[7] = fmaf(wk, v1[k].w, acc[7]);
+    }
+  }
+  const float inv = 1.f / sum;  // sum >= 1: the largest weight is 2^0
+  uint32_t pk[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * k] * inv, acc[2 * k + 1] * inv);
+    pk[k] = *reinterpret_cast<uint32_t*>(&h2);
+  }
+  __nv_bfloat16* olat = static_cast<__nv_bfloat16*>(p.q);
+  *reinterpret_cast<uint4*>(olat + rr * p.r + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+}
+
+// ---------------------------------------------------------------------------
+// up-projection: out[row, h, :] = o_lat[row, h, :] . W_UV[h] (the shard
+// outputs of TPLA are summed by contracting over all r latent columns).
+// grid (H, ceil(rows / 64)); block 256.
 // Shared memory: W_UV[h] [K = 512][M = 128] as 2 MN-major groups of 64 output
-// columns (64 KB each); o_lat [N][512] bf16 as 8 K-major chunks.
+// columns (64 KB each); o_lat rows [N][512] bf16 as 8 K-major chunks (TMA).
 // ---------------------------------------------------------------------------
 struct UprojSmem {
   static constexpr int kMaxRows = 64;                  // query rows per CTA
   static constexpr uint32_t w = 0;                     // 128 KB
   static constexpr uint32_t x = 131072;                // 8 x N x 128 B
-  static constexpr uint32_t lse = x + 8 * kMaxRows * 128;  // float [N][2] totals, int64 [N][2] slot range
-  static constexpr uint32_t bars = lse + kMaxRows * 2 * 4 + kMaxRows * 2 * 8;
+  static constexpr uint32_t bars = x + 8 * kMaxRows * 128;
   static constexpr uint32_t misc = bars + 64;
   static constexpr uint32_t alloc = misc + 64 + 1024;
 };
 
-template <int S>
 __global__ void __launch_bounds__(kThreads, 1)
-    uproj_tc_kernel(const __grid_constant__ CUtensorMap tm_wuv, RunParams p, int n_pad) {
+    uproj_tc_kernel(const __grid_constant__ CUtensorMap tm_wuv,
+                    const __grid_constant__ CUtensorMap tm_olat, RunParams p, int n_pad) {
   using namespace ptx;
   extern __shared__ uint8_t smem_raw[];
-  if (!*p.lengths_ok) return;
+  if (threadIdx.x == 0) MLA_HG_TRACE(1, 0);
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
@@ -173,98 +277,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int row0 = blockIdx.y * UprojSmem::kMaxRows;
   const int nrows = min(UprojSmem::kMaxRows, nbt - row0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar_full = base + UprojSmem::bars, bar_done = bar_full + 8;
+  const uint32_t bar_w = base + UprojSmem::bars, bar_x = bar_w + 8, bar_done = bar_w + 16;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(gbase + UprojSmem::misc);
-  float* lse_tot = reinterpret_cast<float*>(gbase + UprojSmem::lse);  // [N][S]
-  int64_t* seg = reinterpret_cast<int64_t*>(gbase + UprojSmem::lse + UprojSmem::kMaxRows * 2 * 4);
   if (threadIdx.x == 0) {
-    mbar_init(bar_full, 1);
+    mbar_init(bar_w, 1);
+    mbar_init(bar_x, 1);
     mbar_init(bar_done, 1);
     fence_mbarrier_init_cluster();
+    // the weights do not depend on the previous kernels: fetch them at once
     prefetch_tmap(&tm_wuv);
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-                 :: "r"(bar_full), "r"(131072u) : "memory");
+    prefetch_tmap(&tm_olat);
+    mbar_arrive_expect_tx_local(bar_w, 131072u);
     for (int j = 0; j < 2; ++j)      // output columns [64 j, 64 j + 64)
       for (int k = 0; k < 2; ++k)    // latent rows [256 k, 256 k + 256)
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-            :: "r"(base + UprojSmem::w + 65536 * j + 32768 * k),
-               "l"(reinterpret_cast<uint64_t>(&tm_wuv)), "r"(64 * j), "r"(h * p.r + 256 * k),
-               "r"(bar_full) : "memory");
+        tma_load_2d(base + UprojSmem::w + 65536 * j + 32768 * k, &tm_wuv, 64 * j, h * p.r + 256 * k,
+                    bar_w);
   }
   __syncwarp();
   if (warp == 0) {
     tmem_alloc<1>(base + UprojSmem::misc, 128);
     tmem_relinquish<1>();
   }
-  // per-row log2-sum-exp totals over the row's split segments (one warp per row)
-  const int64_t G = p.cum[p.B];
-  for (int i = warp; i < n_pad; i += kThreads / 32) {
-    const int bt = row0 + i;
-    if (i >= nrows) continue;
-    const int b = bt / p.Lq, t = bt % p.Lq, row = t * p.H + h;
-    const int64_t w_lo = page_owner(p.cum[b], G, p.W);
-    const int64_t w_hi = page_owner(p.cum[b + 1] - 1, G, p.W);
-    for (int s = 0; s < S; ++s) {
-      float mx = -INFINITY;
-      for (int64_t w = w_lo + lane; w <= w_hi; w += 32)
-        mx = fmaxf(mx, p.lse_part[((w + b) * p.rows + row) * S + s]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float sum = 0.f;
-      for (int64_t w = w_lo + lane; w <= w_hi; w += 32)
-        sum += exp2f(p.lse_part[((w + b) * p.rows + row) * S + s] - mx);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane == 0) lse_tot[i * S + s] = mx + log2f(sum);
-    }
-    if (lane == 0) {
-      seg[2 * i] = w_lo;
-      seg[2 * i + 1] = w_hi;
-    }
-  }
-  __syncthreads();
-  // o_lat rows -> bf16 B operand, K-major 128B swizzle: row i, latent column c
-  // in chunk c / 64, 16-byte unit (c % 64) / 8
-  const int rs = p.r / S;
-  for (int idx = threadIdx.x; idx < n_pad * 64; idx += blockDim.x) {
-    const int i = idx >> 6, unit = idx & 63;       // unit = 8 latent columns
-    const int c0 = unit * 8;
-    float a[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] = 0.f;
-    if (i < nrows) {
-      const int bt = row0 + i;
-      const int b = bt / p.Lq, t = bt % p.Lq, row = t * p.H + h, s = c0 / rs;
-      const float tot = lse_tot[i * S + s];
-      for (int64_t w = seg[2 * i]; w <= seg[2 * i + 1]; ++w) {
-        const int64_t slot = w + b;
-        const float wt = exp2f(p.lse_part[(slot * p.rows + row) * S + s] - tot);
-        const float4* src = reinterpret_cast<const float4*>(p.o_part + (slot * p.rows + row) * (int64_t)p.r + c0);
-        const float4 v0 = src[0], v1 = src[1];
-        a[0] = fmaf(wt, v0.x, a[0]); a[1] = fmaf(wt, v0.y, a[1]);
-        a[2] = fmaf(wt, v0.z, a[2]); a[3] = fmaf(wt, v0.w, a[3]);
-        a[4] = fmaf(wt, v1.x, a[4]); a[5] = fmaf(wt, v1.y, a[5]);
-        a[6] = fmaf(wt, v1.z, a[6]); a[7] = fmaf(wt, v1.w, a[7]);
-      }
-    }
-    uint32_t pk[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      __nv_bfloat162 h2 = __floats2bfloat162_rn(a[2 * k], a[2 * k + 1]);
-      pk[k] = *reinterpret_cast<uint32_t*>(&h2);
-    }
-    const int chunk = unit >> 3, u16 = unit & 7;
-    *reinterpret_cast<uint4*>(gbase + UprojSmem::x + chunk * n_pad * 128 + sw128(i, u16)) =
-        make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  if (threadIdx.x == 0) {
-    if (mbar_wait<false>(bar_full, 0)) {
+  grid_launch_dependents();
+  grid_dependency_wait();  // o_lat of the combine kernel
+  const bool run = *p.lengths_ok != 0;
+  if (run && threadIdx.x == 0) {
+    mbar_arrive_expect_tx_local(bar_x, 8 * n_pad * 128);
+    for (int kc = 0; kc < 8; ++kc)  // o_lat[row0 .., h, 64 kc .. +64]
+      tma_load_3d(base + UprojSmem::x + kc * n_pad * 128, &tm_olat, 64 * kc, h, row0, bar_x);
+    if (mbar_wait(bar_w, 0) && mbar_wait(bar_x, 0)) {
+      MLA_HG_TRACE(1, 1);
       tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(128, n_pad, 1, 0);
       const uint64_t a0 = smem_desc_sw128(base + UprojSmem::w, 65536, 1024);
@@ -280,8 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncwarp();
-  if (warp < 4) {
-    const bool done = mbar_wait<false>(bar_done, 0);
+  if (run && warp < 4) {
+    const bool done = mbar_wait(bar_done, 0);
+    if (threadIdx.x == 0) MLA_HG_TRACE(1, 2);
     if (__all_sync(0xffffffffu, done)) {
       tc_fence_after();
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
@@ -303,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc<1>(tbase, 128);
+  if (threadIdx.x == 0) MLA_HG_TRACE(1, 3);
 }
 
 // 2-D bf16 row-major [rows, cols] with a (64 columns x box_rows) 128B-swizzled box.
@@ -318,14 +366,31 @@ inline bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t co
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 [d2][d1][d0] (d0 contiguous) with a (64 x 1 x box2) 128B-swizzled box:
+// rows (d2) of one d1 index, 64 columns at a time.
+inline bool make_map3(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint32_t box2) {
+  tc::EncodeTiledFn enc = tc::encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d0, (cuuint64_t)d1, (cuuint64_t)d2};
+  cuuint64_t strides[2] = {(cuuint64_t)d0 * 2, (cuuint64_t)d0 * d1 * 2};
+  cuuint32_t box[3] = {64, 1, box2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline int pad16(int n) { return (n + 15) / 16 * 16; }
+
+
 
 }  // namespace hg
 
 // absorb on tensor cores (bf16, d_nope = 128, r = 512); also scans the lengths
 inline cudaError_t launch_absorb_tc(const RunParams& p, cudaStream_t stream) {
   const int nbt = p.B * p.Lq;
-  const int n_pad = hg::pad16(nbt < hg::kMaxN ? nbt : hg::kMaxN);
+  const int n_pad = hg::pad16(nbt < hg::kAbsorbMaxN ? nbt : hg::kAbsorbMaxN);
   CUtensorMap tm_wuk, tm_qn;
   if (!hg::make_map(&tm_wuk, p.w_uk, (uint64_t)p.H * p.dn, (uint64_t)p.r, 128)) return cudaErrorInvalidValue;
   if (!hg::make_map(&tm_qn, p.q_nope, (uint64_t)nbt, (uint64_t)p.H * p.dn, (uint32_t)n_pad))
@@ -333,32 +398,33 @@ inline cudaError_t launch_absorb_tc(const RunParams& p, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(hg::absorb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)hg::AbsorbSmem::alloc);
   if (e != cudaSuccess) return e;
-  const dim3 grid(p.H, p.r / 128, (nbt + hg::kMaxN - 1) / hg::kMaxN);
-  hg::absorb_tc_kernel<<<grid, hg::kThreads, hg::AbsorbSmem::alloc, stream>>>(tm_wuk, tm_qn, p, n_pad);
-  return cudaGetLastError();
+  const dim3 grid(p.H, (nbt + hg::kAbsorbMaxN - 1) / hg::kAbsorbMaxN);
+  return launch_dependent(hg::absorb_tc_kernel, grid, dim3(hg::kThreads), hg::AbsorbSmem::alloc,
+                              stream, tm_wuk, tm_qn, p, n_pad);
 }
 
-// combine + up-projection on tensor cores (bf16, r = 512, d_v = 128)
-inline cudaError_t launch_uproj_tc(const RunParams& p, cudaStream_t stream) {
+// split merge (bf16 o_lat into the query buffer) + up-projection on tensor
+// cores (bf16, r = 512, d_v = 128)
+inline cudaError_t launch_combine_tc(const RunParams& p, cudaStream_t stream) {
   const int nbt = p.B * p.Lq;
+  const int64_t items = (int64_t)nbt * p.H * (p.r / 8);
+  const dim3 gm((unsigned)((items + hg::kMergeThreads - 1) / hg::kMergeThreads));
+  cudaError_t e = p.S == 1
+      ? launch_dependent(hg::merge_lat_kernel<1>, gm, dim3(hg::kMergeThreads), 0, stream, p)
+      : launch_dependent(hg::merge_lat_kernel<2>, gm, dim3(hg::kMergeThreads), 0, stream, p);
+  if (e != cudaSuccess) return e;
   const int rows_cta = hg::UprojSmem::kMaxRows;
   const int n_pad = hg::pad16(nbt < rows_cta ? nbt : rows_cta);
-  CUtensorMap tm_wuv;
+  CUtensorMap tm_wuv, tm_olat;
   if (!hg::make_map(&tm_wuv, p.w_uv, (uint64_t)p.H * p.r, (uint64_t)p.dv, 256)) return cudaErrorInvalidValue;
+  if (!hg::make_map3(&tm_olat, p.q, (uint64_t)p.r, (uint64_t)p.H, (uint64_t)nbt, (uint32_t)n_pad))
+    return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(hg::uproj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)hg::UprojSmem::alloc);
+  if (e != cudaSuccess) return e;
   const dim3 grid(p.H, (nbt + rows_cta - 1) / rows_cta);
-  cudaError_t e;
-  if (p.S == 1) {
-    e = cudaFuncSetAttribute(hg::uproj_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)hg::UprojSmem::alloc);
-    if (e != cudaSuccess) return e;
-    hg::uproj_tc_kernel<1><<<grid, hg::kThreads, hg::UprojSmem::alloc, stream>>>(tm_wuv, p, n_pad);
-  } else {
-    e = cudaFuncSetAttribute(hg::uproj_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)hg::UprojSmem::alloc);
-    if (e != cudaSuccess) return e;
-    hg::uproj_tc_kernel<2><<<grid, hg::kThreads, hg::UprojSmem::alloc, stream>>>(tm_wuv, p, n_pad);
-  }
-  return cudaGetLastError();
+  return launch_dependent(hg::uproj_tc_kernel, grid, dim3(hg::kThreads), hg::UprojSmem::alloc,
+                              stream, tm_wuv, tm_olat, p, n_pad);
 }
 
 }  // namespace mla
