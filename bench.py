@@ -111,17 +111,34 @@ def recorded_traffic(workload, kernel):
 # clocks sampled during the timed region
 # ----------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU while the timed region
+    runs: NVML queries from a thread every 5 ms (read-only), or nvidia-smi
+    -lms 50 where NVML is not available."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
-        self.lines = []
+        self.rows = []  # (time, sm_mhz, max_mhz, power_w, set of reasons)
         self.proc = None
         self.thread = None
+        self.stop_flag = threading.Event()
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
+            self.nvml = (pynvml, h)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -130,15 +147,41 @@ class ClockSampler:
         except OSError:
             self.proc = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
         time.sleep(0.3)
 
-    def _read(self):
+    def _poll_nvml(self):
+        nv, h = self.nvml
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                mask = int(get_reasons(h))
+                rs = {name for name, bit in self.REASONS if mask & bit}
+                self.rows.append((time.time(), sm, self.max_mhz, pw, rs))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def _read_smi(self):
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
         for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            parts = [x.strip() for x in line.strip().split(",")]
+            if len(parts) < 10:
+                continue
+            rs = {name for (name, _), val in zip(self.REASONS, parts[6:10])
+                  if val.lower().startswith("active")}
+            self.rows.append((time.time(), num(parts[2]), num(parts[3]), num(parts[4]), rs))
 
     def stop(self):
+        self.stop_flag.set()
         if self.proc:
             self.proc.terminate()
             try:
@@ -149,35 +192,19 @@ class ClockSampler:
             self.thread.join(timeout=5)
 
     def summary(self, t0, t1):
-        rows = []
-        for ts, line in self.lines:
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 10:
-                continue
-            rows.append((ts, parts))
-        inside = [p for ts, p in rows if t0 <= ts <= t1]
+        inside = [r for r in self.rows if t0 <= r[0] <= t1]
         if not inside:
-            after = [p for ts, p in rows if ts >= t0]
-            inside = after[:1]
+            inside = [r for r in self.rows if r[0] >= t0][:1]
         if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(p[2]) for p in inside if num(p[2]) is not None]
+        sm = [r[1] for r in inside if r[1] is not None]
         reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for p in inside:
-            for name, val in zip(names, p[6:10]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
+        for r in inside:
+            reasons |= r[4]
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": num(inside[0][3]), "reasons": sorted(reasons),
-                "power_w_max": max((num(p[4]) or 0.0) for p in inside),
-                "samples": len(inside)}
+                "sm_max_mhz": inside[0][2], "reasons": sorted(reasons),
+                "power_w_max": max((r[3] or 0.0) for r in inside),
+                "samples": len(inside), "source": "nvml" if self.nvml else "nvidia-smi"}
 
 
 # ----------------------------------------------------------------------------
@@ -390,6 +417,7 @@ def main():
         step()
     t_stop.record(stream)
     torch.cuda.synchronize(device)
+    w_head = time.time()
     # the decode kernel alone: events recorded on the launch stream around it
     Kd = min(K, 200)
     drv = DriverEvents()
@@ -494,7 +522,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "us_per_step": e2e_ms / Ke * 1e3, "steps": Ke},
         "gpu_launches": info.launches_per_run * K,
-        "clocks": sampler.summary(w0, w1),
+        "clocks": sampler.summary(w0, w_head),
     }
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
