@@ -261,6 +261,28 @@ def init_dist(world):
     return dist
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest value of x over all ranks (each rank times its own GPU)."""
+    if not dist:
+        return x
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, bytes_per_rank: float, ms_per_step: float) -> float:
+    """GB/s of the whole job: every rank processes its own full batch (weak
+    scaling, replicas), timed by the slowest rank."""
+    return world * bytes_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
+def emit(line: dict, rank: int) -> None:
+    """Rank 0 alone prints the JSON line."""
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------
 # oracle timing (cpu_baseline and the reference arm)
 # ----------------------------------------------------------------------------
@@ -432,10 +454,7 @@ def main():
     elapsed_ms = t_start.elapsed_time(t_stop)
     decode_ms = [drv.elapsed_ms(a, b) for a, b in ev]
     drv.destroy()
-    if dist:
-        t = torch.tensor([elapsed_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, device)
     status = plan.read_status()
     if status != 0:
         raise SystemExit(f"device status after timing: {M.mla_status_string(status)}")
@@ -466,14 +485,11 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, device)
 
     ms_step = elapsed_ms / K
-    value = world * work["cache_bytes"] / (ms_step * 1e-3) / 1e9
-    e2e_value = world * work["cache_bytes"] / (e2e_ms / Ke * 1e-3) / 1e9
+    value = whole_job_value(world, work["cache_bytes"], ms_step)
+    e2e_value = whole_job_value(world, work["cache_bytes"], e2e_ms / Ke)
     info = plan.info
     kname = "tcgen05" if info.kernel == M.MLA_KERNEL_TCGEN05 else "simt"
     dec_s = statistics.mean(decode_ms) * 1e-3
@@ -551,8 +567,7 @@ def main():
             "sample": f"{len(pairs)} seeded (sequence, head) pairs at full length, fp64 numpy, "
                       f"scaled by their share of the step's (token x head) work; {dt:.1f} s"}
         line["parity_sample"] = compare_sample(out.cpu(), outs, pairs, wl.dtype)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    emit(line, rank)
     plan.close()
     if dist:
         dist.destroy_process_group()
