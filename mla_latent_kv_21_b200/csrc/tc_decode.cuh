@@ -85,7 +85,7 @@ struct Smem {
   // float [2][S][128] row max (double-buffered by group parity) + [S][128] l
   static constexpr uint32_t xch = p + S * kPBytes;
   static constexpr uint32_t bars = xch + 3 * S * 128 * 4;
-  static constexpr uint32_t nbars = 40;
+  static constexpr uint32_t nbars = 48;
   static constexpr uint32_t misc = bars + nbars * 8;  // tmem slot, abort flag
   static_assert(Cfg<S>::kQkSlots <= 6 && Cfg<S>::kVSlots <= 6, "barrier arrays hold 6 slots");
   static constexpr uint32_t total = misc + 64;
@@ -94,7 +94,7 @@ struct Smem {
 
 // barrier indices (leader = only the leader CTA's copy is used)
 enum : int {
-  B_Q_FULL = 0,       // leader, count 2 (+tx)
+  B_Q_FULL = 0,       // (unused: the query arrives chunk by chunk, B_QC_FULL)
   B_QK_FULL = 1,      // [6] leader, count 2 (+tx)
   B_V_FULL = 7,       // [6] leader, count 2 (+tx)
   B_S_FREE = 13,      // [2] leader, count 8 (4 softmax warps x 2 CTAs)
@@ -108,7 +108,8 @@ enum : int {
   B_FINAL_PV = 33,    // leader, count 1
   B_P_FREE_LO = 34,   // both, count 1: PV is done with P chunks 0, 1 (group pages 0, 1)
   B_P_FREE_HI = 35,   // both, count 1: PV is done with P chunks 2, 3
-  B_COUNT = 36
+  B_QC_FULL = 36,     // [9] leader, count 2 (+tx): query chunk k of the current segment
+  B_COUNT = 45
 };
 
 // Optional event trace (compile with -DMLA_TRACE): SM clock of per-group events
@@ -241,7 +242,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     uint32_t counts[B_COUNT];
     for (int i = 0; i < B_COUNT; ++i) counts[i] = 1;
-    counts[B_Q_FULL] = 2;
+
+    for (int i = 0; i < kChunks; ++i) counts[B_QC_FULL + i] = 2;
     for (int i = 0; i < 6; ++i) counts[B_QK_FULL + i] = 2;
     for (int i = 0; i < 6; ++i) counts[B_V_FULL + i] = 2;
     counts[B_S_FREE] = counts[B_S_FREE + 1] = 8;
@@ -296,19 +298,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool have = g.init(p, w);
       uint32_t cc = 0;  // chunk counter over all groups
       for (int gi = 0; have && ok; ++gi) {
-        if (g.first) {
-          if (gi > 0) {
-            // QK of the previous group (the previous segment's last) must be
-            // done with Q before it is overwritten
-            const int j = gi - 1;
-            ok = mbar_wait(bar(B_S_FULL + j % C::kSBufs), (j / C::kSBufs) & 1);
-            if (!ok) break;
-          }
-          expect_leader(B_Q_FULL, kQBytes);
-          const int y = g.b * p.rows + 64 * (int)rank;
-          for (int k = 0; k < kChunks; ++k)
-            tma_load_2d_pair(base + L::q + k * kQChunkBytes, &tm_q, 64 * k, y, leader_bar(B_Q_FULL));
-        }
+        const int yq = g.b * p.rows + 64 * (int)rank;  // this CTA's query rows of the segment
         const int y0 = page_row(g.b, g.page + 2 * (int)rank, 2 * (int)rank < g.npages);
         const int y1 = page_row(g.b, g.page + 2 * (int)rank + 1, 2 * (int)rank + 1 < g.npages);
         MLA_TRACE_EV(w, rank, EV_LOAD, gi);
@@ -317,6 +307,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (cc >= (uint32_t)C::kQkSlots)
             ok = mbar_wait(bar(B_QK_FREE + slot), ((cc / C::kQkSlots) - 1) & 1);
           if (!ok) break;
+          if (g.first) {
+            // New segment: reload query chunk kc. Its last reader, chunk kc of
+            // the previous group (9 items back), is done: the QK issuer
+            // consumes items in order and item cc - kQkSlots has been released.
+            expect_leader(B_QC_FULL + kc, kQChunkBytes);
+            tma_load_2d_pair(base + L::q + kc * kQChunkBytes, &tm_q, 64 * kc, yq,
+                             leader_bar(B_QC_FULL + kc));
+          }
           expect_leader(B_QK_FULL + slot, kSlotBytes);
           const uint32_t dst = base + L::qk + slot * kSlotBytes;
           tma_load_2d_pair(dst, &tm_kv, 64 * kc, y0, leader_bar(B_QK_FULL + slot));
@@ -371,7 +369,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       GroupCursor g;
       bool have = g.init(p, w);
       for (int gi = 0; have && ok; ++gi) {
-        if (g.first) ok = mbar_wait(bar(B_Q_FULL), g.seg & 1);
         const int sb = gi % C::kSBufs;
         if (ok && gi >= C::kSBufs) ok = mbar_wait(bar(B_S_FREE + sb), ((gi / C::kSBufs) - 1) & 1);
         if (!ok) break;
@@ -379,7 +376,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t s_tmem = tbase + sb * 128 * S;
         for (int kc = 0; kc < kChunks && ok; ++kc, ++cc) {
           const int slot = cc % C::kQkSlots;
-          ok = mbar_wait(bar(B_QK_FULL + slot), (cc / C::kQkSlots) & 1);
+          if (g.first) ok = mbar_wait(bar(B_QC_FULL + kc), g.seg & 1);  // this segment's query chunk
+          ok = ok && mbar_wait(bar(B_QK_FULL + slot), (cc / C::kQkSlots) & 1);
           if (!ok) break;
           MLA_TRACE_CHUNK(w, 0, 1, cc);
           tc_fence_after();
@@ -515,18 +513,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (ok && lane == 0) arrive_leader(B_S_FREE + sb);
         }
+        // masked keys (past the group or the causal limit) become -inf: they
+        // drop out of the max and 2^-inf = 0 in the sum and in P
+        if (nvis < 128) {
+#pragma unroll
+          for (int j = 0; j < 128; ++j)
+            if (j >= nvis) r[j] = 0xff800000u;
+        }
         float mx0 = -INFINITY, mx1 = -INFINITY;
         if (ok) {
-          if (nvis >= 128) {
 #pragma unroll
-            for (int j = 0; j < 128; j += 2) {
-              mx0 = fmaxf(mx0, __uint_as_float(r[j]));
-              mx1 = fmaxf(mx1, __uint_as_float(r[j + 1]));
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 128; ++j)
-              if (j < nvis) mx0 = fmaxf(mx0, __uint_as_float(r[j]));
+          for (int j = 0; j < 128; j += 2) {
+            mx0 = fmaxf(mx0, __uint_as_float(r[j]));
+            mx1 = fmaxf(mx1, __uint_as_float(r[j + 1]));
           }
         }
         const float mt_own = fmaxf(mx0, mx1) * p.scale_log2;
@@ -542,37 +541,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (rescale) alpha = ex2_approx(m[s] - mu);
         m[s] = mu;
         // P = 2^(score * scale - m) in bf16 pairs, row sum in four partial sums
+        // (a row that has seen no key yet keeps m = -inf, all its scores are
+        // -inf and P = 0)
         uint32_t pk[64];
         float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
-        if (ok && mu != -INFINITY) {
-          if (nvis >= 128) {
+        const float nmu = mu == -INFINITY ? 0.f : -mu;
 #pragma unroll
-            for (int j = 0; j < 128; j += 4) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, -mu));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, -mu));
-              const float p2 = ex2_approx(fmaf(__uint_as_float(r[j + 2]), p.scale_log2, -mu));
-              const float p3 = ex2_approx(fmaf(__uint_as_float(r[j + 3]), p.scale_log2, -mu));
-              ps0 += p0; ps1 += p1; ps2 += p2; ps3 += p3;
-              __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
-              __nv_bfloat162 h1 = __floats2bfloat162_rn(p2, p3);
-              pk[j >> 1] = *reinterpret_cast<uint32_t*>(&h0);
-              pk[(j >> 1) + 1] = *reinterpret_cast<uint32_t*>(&h1);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 128; j += 2) {
-              float p0 = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, -mu));
-              float p1 = ex2_approx(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, -mu));
-              p0 = j < nvis ? p0 : 0.f;
-              p1 = j + 1 < nvis ? p1 : 0.f;
-              ps0 += p0; ps1 += p1;
-              __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
-              pk[j >> 1] = *reinterpret_cast<uint32_t*>(&h0);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) pk[j] = 0u;
+        for (int j = 0; j < 128; j += 4) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, nmu));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, nmu));
+          const float p2 = ex2_approx(fmaf(__uint_as_float(r[j + 2]), p.scale_log2, nmu));
+          const float p3 = ex2_approx(fmaf(__uint_as_float(r[j + 3]), p.scale_log2, nmu));
+          ps0 += p0; ps1 += p1; ps2 += p2; ps3 += p3;
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(p2, p3);
+          pk[j >> 1] = *reinterpret_cast<uint32_t*>(&h0);
+          pk[(j >> 1) + 1] = *reinterpret_cast<uint32_t*>(&h1);
         }
         l[s] = l[s] * alpha + ((ps0 + ps1) + (ps2 + ps3));
         if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PASS2, gi);
