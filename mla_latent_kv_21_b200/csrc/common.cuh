@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <mutex>
 #include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -114,6 +115,25 @@ template <typename T> __device__ __forceinline__ T from_float(float x);
 template <> __device__ __forceinline__ float from_float<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device) and
+// remembers it, so that repeated runs (and runs captured into a CUDA graph)
+// make no further attribute calls.
+inline cudaError_t ensure_smem_limit(const void* func, int bytes) {
+  struct Entry { const void* func; int dev; int bytes; };
+  static Entry table[256];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (table[i].func == func && table[i].dev == dev && table[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && used < 256) table[used++] = Entry{func, dev, bytes};
+  return e;
 }
 
 // Launch with programmatic stream serialization: the kernel may start while

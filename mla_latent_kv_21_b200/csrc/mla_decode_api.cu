@@ -251,8 +251,7 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* 
     const dim3 gd(p.W, (p.rows + kSimtRowGroup - 1) / kSimtRowGroup);
     cudaError_t e;
 #define MLA_LAUNCH_DECODE(T, S)                                                              \
-  e = cudaFuncSetAttribute(decode_simt_kernel<T, S>,                                        \
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);          \
+  e = ensure_smem_limit(reinterpret_cast<const void*>(decode_simt_kernel<T, S>), (int)smem);  \
   if (e == cudaSuccess) decode_simt_kernel<T, S><<<gd, kSimtThreads, smem, stream>>>(p);
     if (bf16 && p.S == 1) { MLA_LAUNCH_DECODE(__nv_bfloat16, 1) }
     else if (bf16) { MLA_LAUNCH_DECODE(__nv_bfloat16, 2) }

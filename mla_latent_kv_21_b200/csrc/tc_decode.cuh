@@ -700,14 +700,12 @@ inline cudaError_t launch_tc_decode(const RunParams& p, cudaStream_t stream) {
   if (!tc::make_rows_map(&tm_q, p.q, (uint64_t)p.B * p.rows)) return cudaErrorInvalidValue;
   cudaError_t e;
   if (p.S == 1) {
-    e = cudaFuncSetAttribute(tc::decode_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::Smem<1>::alloc);
+    e = ensure_smem_limit(reinterpret_cast<const void*>(tc::decode_tc_kernel<1>), (int)tc::Smem<1>::alloc);
     if (e != cudaSuccess) return e;
     e = launch_dependent(tc::decode_tc_kernel<1>, dim3(2 * p.W), dim3(tc::kThreads), tc::Smem<1>::alloc,
                          stream, tm_kv, tm_q, p);
   } else {
-    e = cudaFuncSetAttribute(tc::decode_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::Smem<2>::alloc);
+    e = ensure_smem_limit(reinterpret_cast<const void*>(tc::decode_tc_kernel<2>), (int)tc::Smem<2>::alloc);
     if (e != cudaSuccess) return e;
     e = launch_dependent(tc::decode_tc_kernel<2>, dim3(2 * p.W), dim3(tc::kThreads), tc::Smem<2>::alloc,
                          stream, tm_kv, tm_q, p);

@@ -205,9 +205,9 @@ __global__ void __launch_bounds__(kMergeThreads)
   const int64_t lstride = (int64_t)p.rows * S;
   const float* op = p.o_part + (int64_t)row * p.r + c0;
   const int64_t ostride = (int64_t)p.rows * p.r;
-  float mx = -INFINITY;
-  for (int64_t slot = lo; slot <= hi; ++slot) mx = fmaxf(mx, lse[slot * lstride]);
-  float sum = 0.f, acc[8];
+  // one round of loads per 4 segments: the running maximum moves as the
+  // rounds go (a row has at most a few segments, so usually one round)
+  float mx = -INFINITY, sum = 0.f, acc[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) acc[k] = 0.f;
   for (int64_t j0 = lo; j0 <= hi; j0 += 4) {
@@ -226,15 +226,21 @@ __global__ void __launch_bounds__(kMergeThreads)
         v0[k] = v1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
+    const float mn = fmaxf(mx, fmaxf(fmaxf(l[0], l[1]), fmaxf(l[2], l[3])));  // finite: slot j0 exists
+    const float sc = exp2f(mx - mn);  // 0 on the first round
+    sum *= sc;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] *= sc;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const float wk = exp2f(l[k] - mx);
+      const float wk = exp2f(l[k] - mn);
       sum += wk;
       acc[0] = fmaf(wk, v0[k].x, acc[0]); acc[1] = fmaf(wk, v0[k].y, acc[1]);
       acc[2] = fmaf(wk, v0[k].z, acc[2]); acc[3] = fmaf(wk, v0[k].w, acc[3]);
       acc[4] = fmaf(wk, v1[k].x, acc[4]); acc[5] = fmaf(wk, v1[k].y, acc[5]);
       acc[6] = fmaf(wk, v1[k].z, acc[6]); acc[7] = fmaf(wk, v1[k].w, acc[7]);
     }
+    mx = mn;
   }
   const float inv = 1.f / sum;  // sum >= 1: the largest weight is 2^0
   uint32_t pk[4];
@@ -395,8 +401,7 @@ inline cudaError_t launch_absorb_tc(const RunParams& p, cudaStream_t stream) {
   if (!hg::make_map(&tm_wuk, p.w_uk, (uint64_t)p.H * p.dn, (uint64_t)p.r, 128)) return cudaErrorInvalidValue;
   if (!hg::make_map(&tm_qn, p.q_nope, (uint64_t)nbt, (uint64_t)p.H * p.dn, (uint32_t)n_pad))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(hg::absorb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)hg::AbsorbSmem::alloc);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(hg::absorb_tc_kernel), (int)hg::AbsorbSmem::alloc);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.H, (nbt + hg::kAbsorbMaxN - 1) / hg::kAbsorbMaxN);
   return launch_dependent(hg::absorb_tc_kernel, grid, dim3(hg::kThreads), hg::AbsorbSmem::alloc,
@@ -419,8 +424,7 @@ inline cudaError_t launch_combine_tc(const RunParams& p, cudaStream_t stream) {
   if (!hg::make_map(&tm_wuv, p.w_uv, (uint64_t)p.H * p.r, (uint64_t)p.dv, 256)) return cudaErrorInvalidValue;
   if (!hg::make_map3(&tm_olat, p.q, (uint64_t)p.r, (uint64_t)p.H, (uint64_t)nbt, (uint32_t)n_pad))
     return cudaErrorInvalidValue;
-  e = cudaFuncSetAttribute(hg::uproj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)hg::UprojSmem::alloc);
+  e = ensure_smem_limit(reinterpret_cast<const void*>(hg::uproj_tc_kernel), (int)hg::UprojSmem::alloc);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.H, (nbt + rows_cta - 1) / rows_cta);
   return launch_dependent(hg::uproj_tc_kernel, grid, dim3(hg::kThreads), hg::UprojSmem::alloc,
