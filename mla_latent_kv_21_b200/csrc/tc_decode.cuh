@@ -62,9 +62,13 @@ constexpr uint32_t kPBytes = 4 * kPChunkBytes;  // 64 rows x 256 tokens
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;
+// A thread's TMA loads are processed one after another (about 4-5 cycles per
+// 128-byte row on B200); issuing the two boxes of every ring item from two
+// lanes doubles what a producer can stream.
+constexpr int kIssueLanes = 2;
 
 #ifndef MLA_QK_SLOTS
-#define MLA_QK_SLOTS 3
+#define MLA_QK_SLOTS 4
 #endif
 #ifndef MLA_V_SLOTS
 #define MLA_V_SLOTS 4
@@ -74,6 +78,11 @@ struct Cfg {
   static constexpr int kQkSlots = S == 1 ? MLA_QK_SLOTS : 3;
   static constexpr int kVSlots = S == 1 ? MLA_V_SLOTS : 2;
   static constexpr int kSBufs = S == 1 ? 2 : 1;   // S tiles in tensor memory (128 columns each per shard)
+  // One shard: a single 16 KB P buffer holds group pages 0, 1 and then 2, 3
+  // (the second half is written once PV is done with the first), which frees
+  // 16 KB for a fourth QK ring slot. Two shards keep P for all four pages.
+  static constexpr bool kSharedP = S == 1;
+  static constexpr uint32_t kPRegion = kSharedP ? kPBytes / 2 : S * kPBytes;
 };
 
 template <int S>
@@ -83,7 +92,7 @@ struct Smem {
   static constexpr uint32_t v = qk + Cfg<S>::kQkSlots * kSlotBytes;
   static constexpr uint32_t p = v + Cfg<S>::kVSlots * kSlotBytes;
   // float [2][S][128] row max (double-buffered by group parity) + [S][128] l
-  static constexpr uint32_t xch = p + S * kPBytes;
+  static constexpr uint32_t xch = p + Cfg<S>::kPRegion;
   static constexpr uint32_t bars = xch + 3 * S * 128 * 4;
   static constexpr uint32_t nbars = 48;
   static constexpr uint32_t misc = bars + nbars * 8;  // tmem slot, abort flag
@@ -98,7 +107,7 @@ enum : int {
   B_QK_FULL = 1,      // [6] leader, count 2 (+tx)
   B_V_FULL = 7,       // [6] leader, count 2 (+tx)
   B_S_FREE = 13,      // [2] leader, count 8 (4 softmax warps x 2 CTAs)
-  B_P_FULL = 15,      // leader, count 8
+  B_P_FULL = 15,      // leader, count 8: P written (shared P: pages 0, 1 written and O rescaled)
   B_O_FREE = 16,      // leader, count 8
   B_QK_FREE = 17,     // [6] both, count 1 (MMA commit)
   B_V_FREE = 23,      // [6] both, count 1
@@ -106,10 +115,11 @@ enum : int {
   B_PV_DONE = 31,     // both, count 1
   B_FINAL_QK = 32,    // leader, count 1
   B_FINAL_PV = 33,    // leader, count 1
-  B_P_FREE_LO = 34,   // both, count 1: PV is done with P chunks 0, 1 (group pages 0, 1)
-  B_P_FREE_HI = 35,   // both, count 1: PV is done with P chunks 2, 3
+  B_P_FREE_LO = 34,   // both, count 1: PV is done with P of group pages 0, 1
+  B_P_FREE_HI = 35,   // both, count 1: PV is done with P of group pages 2, 3
   B_QC_FULL = 36,     // [9] leader, count 2 (+tx): query chunk k of the current segment
-  B_COUNT = 45
+  B_P_FULL_HI = 45,   // leader, count 4 (shared P: pages 2, 3 written by 2 warps x 2 CTAs)
+  B_COUNT = 46
 };
 
 // Optional event trace (compile with -DMLA_TRACE): SM clock of per-group events
@@ -248,6 +258,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 6; ++i) counts[B_V_FULL + i] = 2;
     counts[B_S_FREE] = counts[B_S_FREE + 1] = 8;
     counts[B_P_FULL] = 8;
+    counts[B_P_FULL_HI] = 4;
     counts[B_O_FREE] = 8;
     for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), counts[i]);
     fence_mbarrier_init_cluster();
@@ -290,24 +301,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // invalid lengths (reported by the length scan): nothing to do
   } else if (warp == 0) {
     // --------------------------------------------- Q and QK chunk producer --
-    if (lane == 0) {
-      prefetch_tmap(&tm_kv);
-      prefetch_tmap(&tm_q);
+    // lanes 0 and 1: lane k loads this CTA's page 2 rank + k of every chunk
+    if (lane < kIssueLanes) {
+      if (lane == 0) {
+        prefetch_tmap(&tm_kv);
+        prefetch_tmap(&tm_q);
+      }
       GroupCursor g;
       bool ok = true;
       bool have = g.init(p, w);
       uint32_t cc = 0;  // chunk counter over all groups
       for (int gi = 0; have && ok; ++gi) {
         const int yq = g.b * p.rows + 64 * (int)rank;  // this CTA's query rows of the segment
-        const int y0 = page_row(g.b, g.page + 2 * (int)rank, 2 * (int)rank < g.npages);
-        const int y1 = page_row(g.b, g.page + 2 * (int)rank + 1, 2 * (int)rank + 1 < g.npages);
-        MLA_TRACE_EV(w, rank, EV_LOAD, gi);
+        const int pg = 2 * (int)rank + lane;            // this lane's page within the group
+        const int y = page_row(g.b, g.page + pg, pg < g.npages);
+        if (lane == 0) MLA_TRACE_EV(w, rank, EV_LOAD, gi);
         for (int kc = 0; kc < kChunks && ok; ++kc, ++cc) {
           const int slot = cc % C::kQkSlots;
           if (cc >= (uint32_t)C::kQkSlots)
             ok = mbar_wait(bar(B_QK_FREE + slot), ((cc / C::kQkSlots) - 1) & 1);
           if (!ok) break;
-          if (g.first) {
+          if (g.first && lane == 1) {
             // New segment: reload query chunk kc. Its last reader, chunk kc of
             // the previous group (9 items back), is done: the QK issuer
             // consumes items in order and item cc - kQkSlots has been released.
@@ -315,11 +329,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tma_load_2d_pair(base + L::q + kc * kQChunkBytes, &tm_q, 64 * kc, yq,
                              leader_bar(B_QC_FULL + kc));
           }
-          expect_leader(B_QK_FULL + slot, kSlotBytes);
-          const uint32_t dst = base + L::qk + slot * kSlotBytes;
-          tma_load_2d_pair(dst, &tm_kv, 64 * kc, y0, leader_bar(B_QK_FULL + slot));
-          tma_load_2d_pair(dst + kSlotBytes / 2, &tm_kv, 64 * kc, y1, leader_bar(B_QK_FULL + slot));
-          MLA_TRACE_CHUNK(w, rank, 0, cc);
+          if (lane == 0) expect_leader(B_QK_FULL + slot, kSlotBytes);
+          tma_load_2d_pair(base + L::qk + slot * kSlotBytes + lane * (kSlotBytes / 2), &tm_kv, 64 * kc, y,
+                           leader_bar(B_QK_FULL + slot));
+          if (lane == 0) MLA_TRACE_CHUNK(w, rank, 0, cc);
         }
         if (ok) have = g.next(p);
       }
@@ -328,7 +341,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------------ V chunk producer --
-    if (lane == 0) {
+    // lanes 0 and 1: lane k loads latent chunk 4 nb + 2 rank + k of every page
+    if (lane < kIssueLanes) {
       GroupCursor g;
       bool ok = true;
       bool have = g.init(p, w);
@@ -342,13 +356,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (vc >= (uint32_t)C::kVSlots)
               ok = mbar_wait(bar(B_V_FREE + slot), ((vc / C::kVSlots) - 1) & 1);
             if (!ok) break;
-            expect_leader(B_V_FULL + slot, kSlotBytes);
-            const uint32_t dst = base + L::v + slot * kSlotBytes;
-            const int chunk = 4 * nb + 2 * (int)rank;
-            tma_load_2d_pair(dst, &tm_kv, 64 * chunk, rows[q], leader_bar(B_V_FULL + slot));
-            tma_load_2d_pair(dst + kSlotBytes / 2, &tm_kv, 64 * (chunk + 1), rows[q],
-                             leader_bar(B_V_FULL + slot));
-            MLA_TRACE_CHUNK(w, rank, 2, vc);
+            if (lane == 0) expect_leader(B_V_FULL + slot, kSlotBytes);
+            const int chunk = 4 * nb + 2 * (int)rank + lane;
+            tma_load_2d_pair(base + L::v + slot * kSlotBytes + lane * (kSlotBytes / 2), &tm_kv, 64 * chunk,
+                             rows[q], leader_bar(B_V_FULL + slot));
+            if (lane == 0) MLA_TRACE_CHUNK(w, rank, 2, vc);
           }
         }
         if (ok) have = g.next(p);
@@ -419,8 +431,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (ok && g.first && g.seg > 0) ok = mbar_wait(bar(B_O_FREE), (g.seg - 1) & 1);
         if (!ok) break;
         MLA_TRACE_EV(w, 0, EV_PV_START, gi);
-        // page-major: P chunks 0, 1 are released half way through
+        // page-major: P of pages 0, 1 is released half way through
         for (int q = 0; q < kGroupPages && ok; ++q) {
+          if (C::kSharedP && q == 2) {
+            ok = mbar_wait(bar(B_P_FULL_HI), gi & 1);  // pages 2, 3 in the shared P buffer
+            if (!ok) break;
+          }
           for (int nb = 0; nb < 2 && ok; ++nb, ++vc) {
             const int shard = S == 2 ? nb : 0;
             const int slot = vc % C::kVSlots;
@@ -428,7 +444,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!ok) break;
             MLA_TRACE_CHUNK(w, 0, 3, vc);
             tc_fence_after();
-            const uint64_t pd = p_desc0 + (uint64_t)((shard * kPBytes + q * kPChunkBytes) >> 4);
+            const int pchunk = C::kSharedP ? (q & 1) : q;
+            const uint64_t pd = p_desc0 + (uint64_t)((shard * kPBytes + pchunk * kPChunkBytes) >> 4);
             const uint64_t vd = v_desc0 + (uint64_t)((slot * kSlotBytes) >> 4);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
@@ -560,50 +577,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         l[s] = l[s] * alpha + ((ps0 + ps1) + (ps2 + ps3));
         if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PASS2, gi);
-        // this warp's P chunks (2 half, 2 half + 1): the previous group's PV
-        // must be done with them
-        if (s == 0 && gi >= 1) wait(half ? B_P_FREE_HI : B_P_FREE_LO, (gi - 1) & 1);
-        if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PBUF_FREE, gi);
-        // rescale this shard's O columns (all 256 for one shard, 128 each for
-        // two) once the previous group's PV is complete
-        if (!g.first && __any_sync(0xffffffffu, rescale)) {
-          wait(B_PV_DONE, (gi - 1) & 1);
-        }
-        if (ok && !g.first && __any_sync(0xffffffffu, rescale)) {
+        auto rescale_o = [&](int c0, int ncols) {
           tc_fence_after();
-          constexpr int kOCols = 256 / S;
 #pragma unroll 1
-          for (int c = 0; c < kOCols; c += 32) {
+          for (int c = c0; c < c0 + ncols; c += 32) {
             uint32_t o[32];
-            tmem_ld32(tbase + lane_off + kTmemO + kOCols * s + c, o);
+            tmem_ld32(tbase + lane_off + kTmemO + c, o);
             tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st32(tbase + lane_off + kTmemO + kOCols * s + c, o);
+            tmem_st32(tbase + lane_off + kTmemO + c, o);
           }
           tmem_wait_st();
-        }
-        if (ok) {
-          // P -> shared memory, K-major 128-byte swizzle: row rloc, tokens
-          // [128 half, +128) = chunks 2 half, 2 half + 1, 16-byte units 0..7 each
-          uint8_t* pbuf = gbase + L::p + s * kPBytes;
+        };
+        // P -> shared memory, K-major 128-byte swizzle: row rloc, this
+        // thread's 128 tokens as two 64-token chunks, 16-byte units 0..7 each
+        auto write_p = [&](uint8_t* chunk0) {
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            uint8_t* chunk = pbuf + (2 * half + t) * kPChunkBytes;
+            uint8_t* chunk = chunk0 + t * kPChunkBytes;
 #pragma unroll
             for (int u = 0; u < 8; ++u)
               *reinterpret_cast<uint4*>(chunk + sw128(rloc, u)) =
                   make_uint4(pk[32 * t + 4 * u], pk[32 * t + 4 * u + 1],
                              pk[32 * t + 4 * u + 2], pk[32 * t + 4 * u + 3]);
           }
+        };
+        if constexpr (C::kSharedP) {
+          // O is rescaled (after the previous group's PV) before this group's
+          // PV adds to it; both halves signal that through B_P_FULL.
+          if (!g.first && __any_sync(0xffffffffu, rescale)) wait(B_PV_DONE, (gi - 1) & 1);
+          if (ok && !g.first && __any_sync(0xffffffffu, rescale)) rescale_o(0, 256);
+          if (half == 0) {
+            // pages 0, 1: the previous group's PV must be done with pages 2, 3
+            if (gi >= 1) wait(B_P_FREE_HI, (gi - 1) & 1);
+          } else {
+            if (ok) tc_fence_before();
+            __syncwarp();
+            if (ok && lane == 0) arrive_leader(B_P_FULL);
+            // pages 2, 3 go where pages 0, 1 were, once this group's PV is done with them
+            wait(B_P_FREE_LO, gi & 1);
+          }
+          if (lq == 0) MLA_TRACE_EV(w, rank, EV_PBUF_FREE, gi);
+          if (ok) {
+            write_p(gbase + L::p);
+            fence_proxy_async_smem();
+            tc_fence_before();
+          }
+          __syncwarp();
+          if (ok && lane == 0) arrive_leader(half == 0 ? B_P_FULL : B_P_FULL_HI);
+        } else {
+          // this warp's P chunks (2 half, 2 half + 1): the previous group's PV
+          // must be done with them
+          if (s == 0 && gi >= 1) wait(half ? B_P_FREE_HI : B_P_FREE_LO, (gi - 1) & 1);
+          if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PBUF_FREE, gi);
+          // rescale this shard's O columns (128 per shard) once the previous
+          // group's PV is complete
+          if (!g.first && __any_sync(0xffffffffu, rescale)) wait(B_PV_DONE, (gi - 1) & 1);
+          if (ok && !g.first && __any_sync(0xffffffffu, rescale)) rescale_o((256 / S) * s, 256 / S);
+          if (ok) write_p(gbase + L::p + s * kPBytes + 2 * half * kPChunkBytes);
         }
       }
-      if (ok) {
-        fence_proxy_async_smem();
-        tc_fence_before();
+      if constexpr (!C::kSharedP) {
+        if (ok) {
+          fence_proxy_async_smem();
+          tc_fence_before();
+        }
+        __syncwarp();
+        if (ok && lane == 0) arrive_leader(B_P_FULL);
       }
-      __syncwarp();
-      if (ok && lane == 0) arrive_leader(B_P_FULL);
       if (lq == 0) MLA_TRACE_EV(w, rank, EV_P_DONE, gi);
 
       if (g.last_of_segment()) {
