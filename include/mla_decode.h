@@ -73,7 +73,9 @@ typedef enum { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype_t;
 typedef enum {
   MLA_KERNEL_AUTO = 0,    /* tcgen05 path where supported, else SIMT */
   MLA_KERNEL_SIMT = 1,    /* CUDA-core fp32 path (all dims; the fp32 path) */
-  MLA_KERNEL_TCGEN05 = 2  /* tensor-core path: bf16, r = 512, d_rope = 64, H*Lq <= 128 */
+  MLA_KERNEL_TCGEN05 = 2, /* tensor-core path: bf16, r = 512, d_rope = 64, H*Lq <= 128 */
+  MLA_KERNEL_TCGEN05_LSPLIT = 3  /* tensor-core path whose CTA pairs split the cached columns
+                                    (each cached byte read once); one latent shard only */
 } mla_kernel_t;
 
 typedef struct {

@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "simt_kernels.cuh"
 #include "tc_decode.cuh"
+#include "tc_decode_ls.cuh"
 #include "tc_head_gemm.cuh"
 
 using namespace mla;
@@ -97,11 +98,14 @@ mla_status_t mla_decode_plan_ex(const mla_dims_t* dims, int32_t batch, const int
   int32_t kernel = o.kernel;
   if (kernel == MLA_KERNEL_AUTO) kernel = tc_supported(*dims) ? MLA_KERNEL_TCGEN05 : MLA_KERNEL_SIMT;
   if (kernel == MLA_KERNEL_TCGEN05 && !tc_supported(*dims)) return MLA_ERR_UNSUPPORTED;
-  if (kernel != MLA_KERNEL_SIMT && kernel != MLA_KERNEL_TCGEN05) return MLA_ERR_INVALID_ARG;
+  if (kernel == MLA_KERNEL_TCGEN05_LSPLIT && !(tc_supported(*dims) && dims->latent_shards == 1))
+    return MLA_ERR_UNSUPPORTED;
+  if (kernel != MLA_KERNEL_SIMT && kernel != MLA_KERNEL_TCGEN05 && kernel != MLA_KERNEL_TCGEN05_LSPLIT)
+    return MLA_ERR_INVALID_ARG;
   int64_t W;
   if (o.num_workers > 0) {
     W = o.num_workers;
-  } else if (kernel == MLA_KERNEL_TCGEN05) {
+  } else if (kernel == MLA_KERNEL_TCGEN05 || kernel == MLA_KERNEL_TCGEN05_LSPLIT) {
     // one CTA pair per worker (a cluster of two SMs); a pair step is one page
     W = std::max<int64_t>(1, std::min<int64_t>(sms / 2, G));
   } else {
@@ -142,7 +146,7 @@ mla_status_t mla_plan_get_info(mla_plan_t plan, mla_plan_info_t* info) {
   info->num_workers = plan->W;
   info->num_split_slots = plan->W + plan->B - 1;
   // tcgen05: absorb, decode, split merge, up-projection; SIMT: absorb, decode, combine
-  info->launches_per_run = plan->kernel == MLA_KERNEL_TCGEN05 ? 4 : 3;
+  info->launches_per_run = plan->kernel == MLA_KERNEL_SIMT ? 3 : 4;
   info->total_pages = plan->G;
   info->workspace_bytes = plan->layout.total;
   return MLA_OK;
@@ -231,7 +235,7 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* 
 
   const bool bf16 = d.dtype == MLA_BF16;
   const int nbt = p.B * p.Lq;
-  const bool tc = plan->kernel == MLA_KERNEL_TCGEN05;
+  const bool tc = plan->kernel == MLA_KERNEL_TCGEN05 || plan->kernel == MLA_KERNEL_TCGEN05_LSPLIT;
   if (tc) {
     if (launch_absorb_tc(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
   } else {
@@ -246,6 +250,8 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* 
   if (ev_start && cudaEventRecord(ev_start, stream) != cudaSuccess) return MLA_ERR_CUDA;
   if (plan->kernel == MLA_KERNEL_TCGEN05) {
     if (launch_tc_decode(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
+  } else if (plan->kernel == MLA_KERNEL_TCGEN05_LSPLIT) {
+    if (launch_ls_decode(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
   } else {
     const size_t smem = simt_decode_smem_bytes(p.r + p.dr, p.S, p.P);
     const dim3 gd(p.W, (p.rows + kSimtRowGroup - 1) / kSimtRowGroup);

@@ -29,6 +29,14 @@ REDUCED = {
 }
 
 
+KERNELS = {"auto": M.MLA_KERNEL_AUTO, "simt": M.MLA_KERNEL_SIMT,
+           "lsplit": M.MLA_KERNEL_TCGEN05_LSPLIT}
+
+
+def _lsplit_ok(wl):
+    return wl.dtype == "bf16" and wl.latent_shards == 1
+
+
 def _cases():
     for name, lens_sets in REDUCED.items():
         for lens in lens_sets:
@@ -36,10 +44,12 @@ def _cases():
 
 
 @pytest.mark.parametrize("name,lens", list(_cases()))
-@pytest.mark.parametrize("kernel", ["auto", "simt"])
+@pytest.mark.parametrize("kernel", ["auto", "simt", "lsplit"])
 def test_reduced_size_parity(cuda_device, name, lens, kernel):
     wl = WORKLOADS[name]
-    k = M.MLA_KERNEL_AUTO if kernel == "auto" else M.MLA_KERNEL_SIMT
+    if kernel == "lsplit" and not _lsplit_ok(wl):
+        pytest.skip("the latent-split kernel takes bf16, one latent shard")
+    k = KERNELS[kernel]
     inputs = generate(wl, seq_lens=lens)
     got, info = run_gpu(wl, inputs, cuda_device, kernel=k)
     ref = oracle_out(wl, inputs)
@@ -55,11 +65,12 @@ FULL_SAMPLES = {
 }
 
 
-@pytest.mark.parametrize("name", list(FULL_SAMPLES))
-def test_full_size_sampled_parity(cuda_device, name):
+@pytest.mark.parametrize("name,kernel", [(n, "auto") for n in FULL_SAMPLES]
+                         + [("deepseek_v3", "lsplit"), ("kimi_k2_mtp", "lsplit")])
+def test_full_size_sampled_parity(cuda_device, name, kernel):
     wl = WORKLOADS[name]
     inputs = generate(wl)
-    got, info = run_gpu(wl, inputs, cuda_device)
+    got, info = run_gpu(wl, inputs, cuda_device, kernel=KERNELS[kernel])
     got = got.double().numpy()
     assert np.isfinite(got).all()
     samples = FULL_SAMPLES[name]
