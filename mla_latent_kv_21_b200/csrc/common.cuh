@@ -8,6 +8,7 @@
 #include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "../../include/mla_decode.h"
 
@@ -47,7 +48,8 @@ MLA_HD int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 //   [4]            int32 lengths_ok (written by the first kernel of a run)
 //   cum            int64 [B + 1] page prefix sums of this run's seq_lens
 //   q              [B * Lq * H, r + d_rope] absorbed query rows (dims.dtype)
-//   o_part         fp32 [slots, rows, r]  per-segment O_lat / l
+//   o_part         [slots, rows, r]  per-segment O_lat / l: fp32 on the SIMT
+//                  path, fp16 on the tensor-core paths (room for fp32 either way)
 //   lse_part       fp32 [slots, rows, S]  per-segment log2-sum-exp per shard
 // ---------------------------------------------------------------------------
 struct WorkspaceLayout {
@@ -94,7 +96,7 @@ struct RunParams {
   int32_t* lengths_ok;
   int64_t* cum;
   void* q;                 // absorbed query rows
-  float* o_part;
+  float* o_part;           // fp32 (SIMT kernels) or fp16 (tensor-core kernels)
   float* lse_part;
   // sizes
   int64_t num_blocks;

@@ -651,6 +651,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (g.last_of_segment()) {
         // ---- segment epilogue: O / l and log2-sum-exp of this segment
         wait(B_PV_DONE, gi & 1);
+        if (lq == 0) MLA_TRACE_EV(w, rank, EV_SYNC1, gi);
         if (ok) tc_fence_after();
 #pragma unroll
         for (int s = 0; s < S; ++s) xl[s * 128 + lq] = l[s];
@@ -665,26 +666,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             p.lse_part[(slot * p.rows + row) * S + s] = lt > 0.f ? m[s] + log2f(lt) : kEmptyLse;
         }
         if (ok) {
-          float* orow = p.o_part + (slot * p.rows + row) * (int64_t)p.r;
+          // O / l goes out as fp16 (the combine kernel reads it back once).
+          // A warp holds 32 consecutive rows; per round it loads 64 columns of
+          // them from tensor memory and transposes the 32 x 128-byte block
+          // through 4 KB of the P buffer (free: this group's PV has completed),
+          // so that each store instruction writes four whole 128-byte row
+          // segments. Swizzle: 16-byte unit u of staged row r sits at u ^ (r & 7).
+          uint8_t* stage = gbase + L::p + (warp & 3) * 4096;
+          const int rbase = 64 * (int)rank + 32 * ((warp & 3) & 1);  // row of lane 0
+          const int j = lane & 7;
+          __half* oh = reinterpret_cast<__half*>(p.o_part);
 #pragma unroll 1
-          for (int c = 0; c < 256; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(tbase + lane_off + kTmemO + c, o);
+          for (int c = 0; c < 256; c += 64) {
+            uint32_t o[64];
+            tmem_ld32(tbase + lane_off + kTmemO + c, *reinterpret_cast<uint32_t(*)[32]>(o));
+            tmem_ld32(tbase + lane_off + kTmemO + c + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
             tmem_wait_ld();
             const int nb = c >> 7;
             const float iv = inv[S == 2 ? nb : 0];
             const int col0 = 256 * nb + 128 * half + (c & 127);
-            if (row_real) {
 #pragma unroll
-              for (int k = 0; k < 32; k += 4)
-                *reinterpret_cast<float4*>(orow + col0 + k) =
-                    make_float4(__uint_as_float(o[k]) * iv, __uint_as_float(o[k + 1]) * iv,
-                                __uint_as_float(o[k + 2]) * iv, __uint_as_float(o[k + 3]) * iv);
+            for (int u = 0; u < 8; ++u) {
+              uint32_t hv[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                __half2 h2 = __floats2half2_rn(__uint_as_float(o[8 * u + 2 * k]) * iv,
+                                               __uint_as_float(o[8 * u + 2 * k + 1]) * iv);
+                hv[k] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+              *reinterpret_cast<uint4*>(stage + lane * 128 + 16 * (u ^ (lane & 7))) =
+                  make_uint4(hv[0], hv[1], hv[2], hv[3]);
             }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = (lane >> 3) + 4 * i;
+              const uint4 v = *reinterpret_cast<const uint4*>(stage + r * 128 + 16 * (j ^ (r & 7)));
+              if (rbase + r < p.rows)
+                *reinterpret_cast<uint4*>(oh + (slot * p.rows + rbase + r) * (int64_t)p.r + col0 + 8 * j) = v;
+            }
+            __syncwarp();
           }
           tc_fence_before();
         }
         named_sync();  // xl and the O reads of all four warps are done
+        if (lq == 0) MLA_TRACE_EV(w, rank, EV_LD0, gi);
         __syncwarp();
         if (ok && lane == 0) arrive_leader(B_O_FREE);
       }

@@ -374,8 +374,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tmem_wait_st();
     };
     // O row / lsum -> partial slot of this segment (this CTA's latent half)
-    auto write_o = [&](int64_t slot, float inv) {
-      float* orow = p.o_part + (slot * p.rows + row) * (int64_t)p.r + col_lat;
+    auto write_o = [&](int64_t slot, float inv) {  // fp16, as the combine kernel reads it
+      __half* orow = reinterpret_cast<__half*>(p.o_part) + (slot * p.rows + row) * (int64_t)p.r + col_lat;
 #pragma unroll 1
       for (int c = 0; c < 256; c += 32) {
         uint32_t o[32];
@@ -383,10 +383,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         if (row_real) {
 #pragma unroll
-          for (int k = 0; k < 32; k += 4)
-            *reinterpret_cast<float4*>(orow + c + k) =
-                make_float4(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv,
-                            __uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
+          for (int k = 0; k < 32; k += 8) {
+            uint32_t hv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __half2 h2 = __floats2half2_rn(__uint_as_float(o[k + 2 * e]) * inv,
+                                             __uint_as_float(o[k + 2 * e + 1]) * inv);
+              hv[e] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            *reinterpret_cast<uint4*>(orow + c + k) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          }
         }
       }
     };

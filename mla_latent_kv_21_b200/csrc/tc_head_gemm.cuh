@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // combine: o_lat = log-sum-exp merge of a row's split partials, per TPLA shard.
 // One thread per (query row, head, 8 latent columns); the 64 threads of a row
-// read each partial row as 2 KB of consecutive bytes. Writes bf16 o_lat
+// read each fp16 partial row as 1 KB of consecutive bytes. Writes bf16 o_lat
 // [B * Lq * H, r] into the absorbed-query buffer, which the decode no longer
 // needs. grid ceil(B * Lq * H * 64 / 256), block 256.
 // ---------------------------------------------------------------------------
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kMergeThreads)
   const int64_t hi = page_owner(p.cum[b + 1] - 1, G, p.W) + b;
   const float* lse = p.lse_part + (int64_t)row * S + s;
   const int64_t lstride = (int64_t)p.rows * S;
-  const float* op = p.o_part + (int64_t)row * p.r + c0;
+  const __half* op = reinterpret_cast<const __half*>(p.o_part) + (int64_t)row * p.r + c0;
   const int64_t ostride = (int64_t)p.rows * p.r;
   // one round of loads per 4 segments: the running maximum moves as the
   // rounds go (a row has at most a few segments, so usually one round)
@@ -212,18 +212,16 @@ __global__ void __launch_bounds__(kMergeThreads)
   for (int k = 0; k < 8; ++k) acc[k] = 0.f;
   for (int64_t j0 = lo; j0 <= hi; j0 += 4) {
     float l[4];
-    float4 v0[4], v1[4];
+    uint4 raw[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int64_t slot = j0 + k;
       if (slot <= hi) {
         l[k] = lse[slot * lstride];
-        const float4* q4 = reinterpret_cast<const float4*>(op + slot * ostride);
-        v0[k] = q4[0];
-        v1[k] = q4[1];
+        raw[k] = *reinterpret_cast<const uint4*>(op + slot * ostride);
       } else {
         l[k] = -INFINITY;
-        v0[k] = v1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        raw[k] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     const float mn = fmaxf(mx, fmaxf(fmaxf(l[0], l[1]), fmaxf(l[2], l[3])));  // finite: slot j0 exists
@@ -235,10 +233,13 @@ __global__ void __launch_bounds__(kMergeThreads)
     for (int k = 0; k < 4; ++k) {
       const float wk = exp2f(l[k] - mn);
       sum += wk;
-      acc[0] = fmaf(wk, v0[k].x, acc[0]); acc[1] = fmaf(wk, v0[k].y, acc[1]);
-      acc[2] = fmaf(wk, v0[k].z, acc[2]); acc[3] = fmaf(wk, v0[k].w, acc[3]);
-      acc[4] = fmaf(wk, v1[k].x, acc[4]); acc[5] = fmaf(wk, v1[k].y, acc[5]);
-      acc[6] = fmaf(wk, v1[k].z, acc[6]); acc[7] = fmaf(wk, v1[k].w, acc[7]);
+      const uint32_t hw[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hw[e]));
+        acc[2 * e] = fmaf(wk, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(wk, f.y, acc[2 * e + 1]);
+      }
     }
     mx = mn;
   }
