@@ -145,8 +145,8 @@ mla_status_t mla_plan_get_info(mla_plan_t plan, mla_plan_info_t* info) {
   info->kernel = plan->kernel;
   info->num_workers = plan->W;
   info->num_split_slots = plan->W + plan->B - 1;
-  // tcgen05: absorb, decode, split merge, up-projection; SIMT: absorb, decode, combine
-  info->launches_per_run = plan->kernel == MLA_KERNEL_SIMT ? 3 : 4;
+  // absorb, decode, combine (split merge fused with the up-projection)
+  info->launches_per_run = 3;
   info->total_pages = plan->G;
   info->workspace_bytes = plan->layout.total;
   return MLA_OK;

@@ -2,7 +2,7 @@
 //
 //   absorb : q_lat[row, :] = q_nope[row, h, :] . W_UK[h]            (K = 128, 512 outputs)
 //            (TransMLA abstract: W_UK is absorbed into the query)
-//   up-proj: out[row, h, :] = o_lat[row, h, :] . W_UV[h]             (K = 512, 128 outputs)
+//   combine: out[row, h, :] = o_lat[row, h, :] . W_UV[h]             (K = 512, 128 outputs)
 //            where o_lat is the log-sum-exp merge of the split partials
 //            (per TPLA shard, then the shards are contracted together, which
 //            sums the shard outputs; TPLA abstract)
@@ -173,95 +173,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// combine: o_lat = log-sum-exp merge of a row's split partials, per TPLA shard.
-// One thread per (query row, head, 8 latent columns); the 64 threads of a row
-// read each fp16 partial row as 1 KB of consecutive bytes. Writes bf16 o_lat
-// [B * Lq * H, r] into the absorbed-query buffer, which the decode no longer
-// needs. grid ceil(B * Lq * H * 64 / 256), block 256.
+// combine: out[row, h, :] = o_lat[row, h, :] . W_UV[h], where o_lat is the
+// log-sum-exp merge of the row's split partials (per TPLA shard; contracting
+// over all r latent columns then sums the shard outputs). One kernel:
+//   1. W_UV[h] (128 KB, [K = 512][M = 128] as 2 MN-major groups of 64 output
+//      columns) is fetched by TMA before the dependency wait, so it overlaps
+//      the tail of the decode kernel;
+//   2. after the wait, the 512 threads merge the fp16 partials of the CTA's
+//      rows (a thread takes a row x 32 latent columns and issues the loads of
+//      all its segments at once) and write bf16 o_lat straight into shared
+//      memory as the K-major B operand (8 chunks of 64 latent columns,
+//      128-byte swizzle), so o_lat never goes to HBM;
+//   3. one thread issues the 32 MMAs (M = 128 outputs, N = rows, K = 512);
+//   4. 4 warps read the accumulator and write the bf16 output rows.
+// grid (H, ceil(rows / 64)); block 512.
 // ---------------------------------------------------------------------------
-constexpr int kMergeThreads = 256;
-
-template <int S>
-__global__ void __launch_bounds__(kMergeThreads)
-    merge_lat_kernel(RunParams p) {
-  using namespace ptx;
-  grid_launch_dependents();
-  grid_dependency_wait();  // the partials of the decode kernel
-  if (!*p.lengths_ok) return;
-  const int units = p.r / 8;
-  const int64_t nitems = (int64_t)p.B * p.Lq * p.H * units;
-  const int64_t idx = (int64_t)blockIdx.x * kMergeThreads + threadIdx.x;
-  if (idx >= nitems) return;
-  const int unit = (int)(idx % units);
-  const int64_t rr = idx / units;                  // (b, t) * H + h
-  const int h = (int)(rr % p.H);
-  const int bt = (int)(rr / p.H);
-  const int b = bt / p.Lq, t = bt % p.Lq, row = t * p.H + h;
-  const int c0 = unit * 8, s = c0 / (p.r / S);
-  const int64_t G = p.cum[p.B];
-  const int64_t lo = page_owner(p.cum[b], G, p.W) + b;
-  const int64_t hi = page_owner(p.cum[b + 1] - 1, G, p.W) + b;
-  const float* lse = p.lse_part + (int64_t)row * S + s;
-  const int64_t lstride = (int64_t)p.rows * S;
-  const __half* op = reinterpret_cast<const __half*>(p.o_part) + (int64_t)row * p.r + c0;
-  const int64_t ostride = (int64_t)p.rows * p.r;
-  // one round of loads per 4 segments: the running maximum moves as the
-  // rounds go (a row has at most a few segments, so usually one round)
-  float mx = -INFINITY, sum = 0.f, acc[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
-  for (int64_t j0 = lo; j0 <= hi; j0 += 4) {
-    float l[4];
-    uint4 raw[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t slot = j0 + k;
-      if (slot <= hi) {
-        l[k] = lse[slot * lstride];
-        raw[k] = *reinterpret_cast<const uint4*>(op + slot * ostride);
-      } else {
-        l[k] = -INFINITY;
-        raw[k] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-    const float mn = fmaxf(mx, fmaxf(fmaxf(l[0], l[1]), fmaxf(l[2], l[3])));  // finite: slot j0 exists
-    const float sc = exp2f(mx - mn);  // 0 on the first round
-    sum *= sc;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) acc[k] *= sc;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float wk = exp2f(l[k] - mn);
-      sum += wk;
-      const uint32_t hw[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hw[e]));
-        acc[2 * e] = fmaf(wk, f.x, acc[2 * e]);
-        acc[2 * e + 1] = fmaf(wk, f.y, acc[2 * e + 1]);
-      }
-    }
-    mx = mn;
-  }
-  const float inv = 1.f / sum;  // sum >= 1: the largest weight is 2^0
-  uint32_t pk[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * k] * inv, acc[2 * k + 1] * inv);
-    pk[k] = *reinterpret_cast<uint32_t*>(&h2);
-  }
-  __nv_bfloat16* olat = static_cast<__nv_bfloat16*>(p.q);
-  *reinterpret_cast<uint4*>(olat + rr * p.r + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-}
-
-// ---------------------------------------------------------------------------
-// up-projection: out[row, h, :] = o_lat[row, h, :] . W_UV[h] (the shard
-// outputs of TPLA are summed by contracting over all r latent columns).
-// grid (H, ceil(rows / 64)); block 256.
-// Shared memory: W_UV[h] [K = 512][M = 128] as 2 MN-major groups of 64 output
-// columns (64 KB each); o_lat rows [N][512] bf16 as 8 K-major chunks (TMA).
-// ---------------------------------------------------------------------------
-struct UprojSmem {
+struct CombineSmem {
   static constexpr int kMaxRows = 64;                  // query rows per CTA
   static constexpr uint32_t w = 0;                     // 128 KB
   static constexpr uint32_t x = 131072;                // 8 x N x 128 B
@@ -270,9 +197,11 @@ struct UprojSmem {
   static constexpr uint32_t alloc = misc + 64 + 1024;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
-    uproj_tc_kernel(const __grid_constant__ CUtensorMap tm_wuv,
-                    const __grid_constant__ CUtensorMap tm_olat, RunParams p, int n_pad) {
+constexpr int kCombineThreads = 512;
+
+template <int S>
+__global__ void __launch_bounds__(kCombineThreads, 1)
+    combine_tc_kernel(const __grid_constant__ CUtensorMap tm_wuv, RunParams p, int n_pad) {
   using namespace ptx;
   extern __shared__ uint8_t smem_raw[];
   if (threadIdx.x == 0) MLA_HG_TRACE(1, 0);
@@ -281,28 +210,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw);
   const int h = blockIdx.x;
   const int nbt = p.B * p.Lq;
-  const int row0 = blockIdx.y * UprojSmem::kMaxRows;
-  const int nrows = min(UprojSmem::kMaxRows, nbt - row0);
+  const int row0 = blockIdx.y * CombineSmem::kMaxRows;
+  const int nrows = min(CombineSmem::kMaxRows, nbt - row0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar_w = base + UprojSmem::bars, bar_x = bar_w + 8, bar_done = bar_w + 16;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(gbase + UprojSmem::misc);
+  const uint32_t bar_w = base + CombineSmem::bars, bar_done = bar_w + 16;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(gbase + CombineSmem::misc);
   if (threadIdx.x == 0) {
     mbar_init(bar_w, 1);
-    mbar_init(bar_x, 1);
     mbar_init(bar_done, 1);
     fence_mbarrier_init_cluster();
     // the weights do not depend on the previous kernels: fetch them at once
     prefetch_tmap(&tm_wuv);
-    prefetch_tmap(&tm_olat);
     mbar_arrive_expect_tx_local(bar_w, 131072u);
     for (int j = 0; j < 2; ++j)      // output columns [64 j, 64 j + 64)
       for (int k = 0; k < 2; ++k)    // latent rows [256 k, 256 k + 256)
-        tma_load_2d(base + UprojSmem::w + 65536 * j + 32768 * k, &tm_wuv, 64 * j, h * p.r + 256 * k,
+        tma_load_2d(base + CombineSmem::w + 65536 * j + 32768 * k, &tm_wuv, 64 * j, h * p.r + 256 * k,
                     bar_w);
   }
   __syncwarp();
   if (warp == 0) {
-    tmem_alloc<1>(base + UprojSmem::misc, 128);
+    tmem_alloc<1>(base + CombineSmem::misc, 128);
     tmem_relinquish<1>();
   }
   tc_fence_before();
@@ -310,18 +237,102 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tslot;
   grid_launch_dependents();
-  grid_dependency_wait();  // o_lat of the combine kernel
+  grid_dependency_wait();  // the partials of the decode kernel
   const bool run = *p.lengths_ok != 0;
+  if (run) {
+    // ---- merge: one item = one row x 32 latent columns (64 bytes of each fp16
+    // partial row; the 16 items of a row read it as 1 KB of consecutive
+    // bytes). Each thread issues all loads of an item's first 4 segments at
+    // once, so the merge costs about two L2 round trips per item.
+    const int64_t G = p.cum[p.B];
+    const int64_t lstride = (int64_t)p.rows * S;
+    const int64_t ostride = (int64_t)p.rows * p.r;
+    const __half* opart = reinterpret_cast<const __half*>(p.o_part);
+    for (int it = threadIdx.x; it < n_pad * 16; it += kCombineThreads) {
+      const int i = it >> 4, slice = it & 15;
+      const int c0 = 32 * slice;
+      uint4 packed[4] = {};  // padding rows stay zero
+      if (i < nrows) {
+        const int bt = row0 + i, b = bt / p.Lq, t = bt % p.Lq, row = t * p.H + h;
+        const int sh = c0 / (p.r / S);
+        const int64_t lo = page_owner(p.cum[b], G, p.W) + b;
+        const int64_t hi = page_owner(p.cum[b + 1] - 1, G, p.W) + b;
+        const float* lse = p.lse_part + (int64_t)row * S + sh;
+        const __half* op = opart + (int64_t)row * p.r + c0;
+        // one round of loads per 4 segments; the running maximum moves as the
+        // rounds go (a row has at most a few segments, so usually one round)
+        float mx = -INFINITY, sum = 0.f, acc[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+        for (int64_t j0 = lo; j0 <= hi; j0 += 4) {
+          float l[4];
+          uint4 v[4][4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int64_t slot = j0 + k;
+            if (slot <= hi) {
+              l[k] = lse[slot * lstride];
+              const uint4* src = reinterpret_cast<const uint4*>(op + slot * ostride);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) v[k][q] = src[q];
+            } else {
+              l[k] = -INFINITY;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) v[k][q] = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+          const float mn = fmaxf(mx, fmaxf(fmaxf(l[0], l[1]), fmaxf(l[2], l[3])));  // slot j0 exists
+          const float sc = exp2f(mx - mn);  // 0 on the first round
+          sum *= sc;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) acc[k] *= sc;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float wk = exp2f(l[k] - mn);
+            sum += wk;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t hw[4] = {v[k][q].x, v[k][q].y, v[k][q].z, v[k][q].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hw[e]));
+                acc[8 * q + 2 * e] = fmaf(wk, f.x, acc[8 * q + 2 * e]);
+                acc[8 * q + 2 * e + 1] = fmaf(wk, f.y, acc[8 * q + 2 * e + 1]);
+              }
+            }
+          }
+          mx = mn;
+        }
+        const float inv = 1.f / sum;  // sum >= 1: the largest weight is 2^0
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[8 * q + 2 * k] * inv, acc[8 * q + 2 * k + 1] * inv);
+            pk[k] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          packed[q] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      // o_lat[row0 + i, h, 8u .. +8] for u = 4 slice + q -> chunk u / 8, row i,
+      // 16-byte unit u % 8 of the 128-byte-swizzled K-major operand
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int u = 4 * slice + q;
+        *reinterpret_cast<uint4*>(gbase + CombineSmem::x + (u >> 3) * n_pad * 128 + sw128(i, u & 7)) = packed[q];
+      }
+    }
+    fence_proxy_async_smem();  // generic writes -> tensor core reads
+  }
+  __syncthreads();
   if (run && threadIdx.x == 0) {
-    mbar_arrive_expect_tx_local(bar_x, 8 * n_pad * 128);
-    for (int kc = 0; kc < 8; ++kc)  // o_lat[row0 .., h, 64 kc .. +64]
-      tma_load_3d(base + UprojSmem::x + kc * n_pad * 128, &tm_olat, 64 * kc, h, row0, bar_x);
-    if (mbar_wait(bar_w, 0) && mbar_wait(bar_x, 0)) {
+    if (mbar_wait(bar_w, 0)) {
       MLA_HG_TRACE(1, 1);
       tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(128, n_pad, 1, 0);
-      const uint64_t a0 = smem_desc_sw128(base + UprojSmem::w, 65536, 1024);
-      const uint64_t b0 = smem_desc_sw128(base + UprojSmem::x, 16, 1024);
+      const uint64_t a0 = smem_desc_sw128(base + CombineSmem::w, 65536, 1024);
+      const uint64_t b0 = smem_desc_sw128(base + CombineSmem::x, 16, 1024);
       for (int ks = 0; ks < 32; ++ks) {  // K = 512 = 32 x 16
         const uint64_t ad = a0 + (uint64_t)(128 * ks);
         const uint64_t bd = b0 + (uint64_t)(((ks >> 2) * n_pad * 128) >> 4) + (uint64_t)(2 * (ks & 3));
@@ -373,21 +384,6 @@ inline bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t co
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D bf16 [d2][d1][d0] (d0 contiguous) with a (64 x 1 x box2) 128B-swizzled box:
-// rows (d2) of one d1 index, 64 columns at a time.
-inline bool make_map3(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
-                      uint32_t box2) {
-  tc::EncodeTiledFn enc = tc::encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)d0, (cuuint64_t)d1, (cuuint64_t)d2};
-  cuuint64_t strides[2] = {(cuuint64_t)d0 * 2, (cuuint64_t)d0 * d1 * 2};
-  cuuint32_t box[3] = {64, 1, box2};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 inline int pad16(int n) { return (n + 15) / 16 * 16; }
 
 
@@ -413,23 +409,19 @@ inline cudaError_t launch_absorb_tc(const RunParams& p, cudaStream_t stream) {
 // cores (bf16, r = 512, d_v = 128)
 inline cudaError_t launch_combine_tc(const RunParams& p, cudaStream_t stream) {
   const int nbt = p.B * p.Lq;
-  const int64_t items = (int64_t)nbt * p.H * (p.r / 8);
-  const dim3 gm((unsigned)((items + hg::kMergeThreads - 1) / hg::kMergeThreads));
-  cudaError_t e = p.S == 1
-      ? launch_dependent(hg::merge_lat_kernel<1>, gm, dim3(hg::kMergeThreads), 0, stream, p)
-      : launch_dependent(hg::merge_lat_kernel<2>, gm, dim3(hg::kMergeThreads), 0, stream, p);
-  if (e != cudaSuccess) return e;
-  const int rows_cta = hg::UprojSmem::kMaxRows;
+  const int rows_cta = hg::CombineSmem::kMaxRows;
   const int n_pad = hg::pad16(nbt < rows_cta ? nbt : rows_cta);
-  CUtensorMap tm_wuv, tm_olat;
+  CUtensorMap tm_wuv;
   if (!hg::make_map(&tm_wuv, p.w_uv, (uint64_t)p.H * p.r, (uint64_t)p.dv, 256)) return cudaErrorInvalidValue;
-  if (!hg::make_map3(&tm_olat, p.q, (uint64_t)p.r, (uint64_t)p.H, (uint64_t)nbt, (uint32_t)n_pad))
-    return cudaErrorInvalidValue;
-  e = ensure_smem_limit(reinterpret_cast<const void*>(hg::uproj_tc_kernel), (int)hg::UprojSmem::alloc);
+  const void* fn = p.S == 1 ? reinterpret_cast<const void*>(hg::combine_tc_kernel<1>)
+                            : reinterpret_cast<const void*>(hg::combine_tc_kernel<2>);
+  cudaError_t e = ensure_smem_limit(fn, (int)hg::CombineSmem::alloc);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.H, (nbt + rows_cta - 1) / rows_cta);
-  return launch_dependent(hg::uproj_tc_kernel, grid, dim3(hg::kThreads), hg::UprojSmem::alloc,
-                              stream, tm_wuv, tm_olat, p, n_pad);
+  return p.S == 1 ? launch_dependent(hg::combine_tc_kernel<1>, grid, dim3(hg::kCombineThreads),
+                                     hg::CombineSmem::alloc, stream, tm_wuv, p, n_pad)
+                  : launch_dependent(hg::combine_tc_kernel<2>, grid, dim3(hg::kCombineThreads),
+                                     hg::CombineSmem::alloc, stream, tm_wuv, p, n_pad);
 }
 
 }  // namespace mla
