@@ -21,22 +21,42 @@ namespace mla {
 //
 // The pages of all sequences are concatenated (sequence b owns global pages
 // [cum[b], cum[b+1]), cum[b] = sum_{i<b} ceil(L_i / P)) and cut into W
-// contiguous page ranges, worker w owning [start(w), start(w+1)) with
-// start(w) = floor(w * G / W). A worker's range meets one or more sequences;
-// each (worker, sequence) intersection is one split segment whose partial
-// result goes to slot w + b. Along the concatenated page order both w and b
-// are non-decreasing and at least one of them grows from one segment to the
-// next, so w + b is strictly increasing: slots are unique, and W + B - 1 slots
-// always suffice whatever the lengths are.
+// contiguous page ranges. A worker's range meets one or more sequences; each
+// (worker, sequence) intersection is one split segment whose partial result
+// goes to slot w + b. Along the concatenated page order both w and b are
+// non-decreasing and at least one of them grows from one segment to the next,
+// so w + b is strictly increasing: slots are unique, and W + B - 1 slots always
+// suffice whatever the lengths are.
+//
+// The cut balances cost, not pages: a worker whose range crosses a sequence
+// boundary writes one more segment partial and reloads the query, which costs
+// about as much as kSegmentCostPages pages. So every boundary takes that many
+// places on a "virtual" page line (page x of sequence b sits at x + c b, and
+// the line is G' = G + c (B - 1) long), the line is cut evenly, at
+// floor(w G' / W), and each cut moves to the first real page at or after it.
 // ---------------------------------------------------------------------------
-MLA_HD int64_t worker_page_start(int64_t w, int64_t G, int64_t W) {
-  return (w * G) / W;
+constexpr int64_t kSegmentCostPages = 4;
+
+MLA_HD int64_t virtual_pages(int64_t G, int64_t B) { return G + kSegmentCostPages * (B - 1); }
+
+// start(w): the first global page of worker w (start(W) = G). cum has B + 1
+// entries, strictly increasing (every sequence has at least one page).
+MLA_HD int64_t worker_page_start(int64_t w, const int64_t* cum, int64_t B, int64_t W) {
+  const int64_t v = (w * virtual_pages(cum[B], B)) / W;
+  int64_t lo = 0, hi = B - 1;  // the last sequence b with cum[b] + c b <= v
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) >> 1;
+    if (cum[mid] + kSegmentCostPages * mid <= v) lo = mid; else hi = mid - 1;
+  }
+  const int64_t x = v - kSegmentCostPages * lo;
+  return x < cum[lo + 1] ? x : cum[lo + 1];  // a cut inside a boundary moves to the next sequence
 }
 
-// The worker whose range holds global page x (0 <= x < G): the largest w with
-// start(w) <= x, i.e. w = ceil((x + 1) * W / G) - 1, clamped to W - 1.
-MLA_HD int64_t page_owner(int64_t x, int64_t G, int64_t W) {
-  int64_t w = ((x + 1) * W + G - 1) / G - 1;
+// The worker whose range holds page x of sequence b: the largest w with
+// start(w) <= x, i.e. with floor(w G' / W) <= x + c b, clamped to W - 1.
+MLA_HD int64_t page_owner(int64_t x, int64_t b, int64_t Gv, int64_t W) {
+  const int64_t xv = x + kSegmentCostPages * b;
+  const int64_t w = ((xv + 1) * W + Gv - 1) / Gv - 1;
   return w < W - 1 ? w : W - 1;
 }
 

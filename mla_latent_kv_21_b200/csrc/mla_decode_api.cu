@@ -154,12 +154,13 @@ mla_status_t mla_plan_get_info(mla_plan_t plan, mla_plan_info_t* info) {
 
 mla_status_t mla_plan_segments(mla_plan_t plan, int32_t* out, int64_t capacity, int64_t* count) {
   if (!plan || !count || capacity < 0 || (capacity > 0 && !out)) return MLA_ERR_INVALID_ARG;
-  const int64_t P = plan->dims.page_size, G = plan->G, W = plan->W;
+  const int64_t P = plan->dims.page_size, W = plan->W;
   std::vector<int64_t> cum(plan->B + 1, 0);
   for (int b = 0; b < plan->B; ++b) cum[b + 1] = cum[b] + ceil_div64(plan->lens[b], P);
   int64_t n = 0;
   for (int64_t w = 0; w < W; ++w) {
-    const int64_t g0 = worker_page_start(w, G, W), g1 = worker_page_start(w + 1, G, W);
+    const int64_t g0 = worker_page_start(w, cum.data(), plan->B, W),
+                  g1 = worker_page_start(w + 1, cum.data(), plan->B, W);
     if (g0 >= g1) continue;
     int b = 0;
     while (cum[b + 1] <= g0) ++b;

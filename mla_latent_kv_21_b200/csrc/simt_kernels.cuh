@@ -141,8 +141,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(RunParams p) 
   float* a_s = l_s + S * kSimtRowGroup;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int w = blockIdx.x, row0 = blockIdx.y * kSimtRowGroup;
-  const int64_t G = p.cum[p.B];
-  const int64_t g0 = worker_page_start(w, G, p.W), g1 = worker_page_start(w + 1, G, p.W);
+  const int64_t g0 = worker_page_start(w, p.cum, p.B, p.W), g1 = worker_page_start(w + 1, p.cum, p.B, p.W);
   if (g0 >= g1) return;
   const T* pool = static_cast<const T*>(p.kv);
   const T* qg = static_cast<const T*>(p.q);
@@ -288,14 +287,14 @@ __global__ void __launch_bounds__(kSimtThreads) combine_simt_kernel(RunParams p)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x, bt0 = blockIdx.y * kCombineRows;
   const int nbt = p.B * p.Lq;
-  const int64_t G = p.cum[p.B];
+  const int64_t Gv = virtual_pages(p.cum[p.B], p.B);
   const int rs = p.r / S;
   if (warp < kCombineRows) {
     const int i = warp, bt = bt0 + i;
     if (bt < nbt) {
       const int b = bt / p.Lq, t = bt % p.Lq, row = t * p.H + h;
-      const int64_t w_lo = page_owner(p.cum[b], G, p.W);
-      const int64_t w_hi = page_owner(p.cum[b + 1] - 1, G, p.W);
+      const int64_t w_lo = page_owner(p.cum[b], b, Gv, p.W);
+      const int64_t w_hi = page_owner(p.cum[b + 1] - 1, b, Gv, p.W);
       for (int s = 0; s < S; ++s) {
         float mx = -INFINITY;
         for (int64_t w = w_lo + lane; w <= w_hi; w += 32)

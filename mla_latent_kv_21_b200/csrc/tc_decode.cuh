@@ -176,9 +176,8 @@ struct GroupCursor {
   __device__ __forceinline__ void set_group() { npages = min(kGroupPages, pe - page); }
   // returns false when the worker has no pages
   __device__ __forceinline__ bool init(const RunParams& p, int w) {
-    const int64_t G = p.cum[p.B];
-    const int64_t g0 = worker_page_start(w, G, p.W);
-    g1 = worker_page_start(w + 1, G, p.W);
+    const int64_t g0 = worker_page_start(w, p.cum, p.B, p.W);
+    g1 = worker_page_start(w + 1, p.cum, p.B, p.W);
     if (g0 >= g1) return false;
     int lo = 0, hi = p.B - 1;
     while (lo < hi) {

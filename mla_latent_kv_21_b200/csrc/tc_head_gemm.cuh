@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kCombineThreads, 1)
     // partial row; the 16 items of a row read it as 1 KB of consecutive
     // bytes). Each thread issues all loads of an item's first 4 segments at
     // once, so the merge costs about two L2 round trips per item.
-    const int64_t G = p.cum[p.B];
+    const int64_t Gv = virtual_pages(p.cum[p.B], p.B);
     const int64_t lstride = (int64_t)p.rows * S;
     const int64_t ostride = (int64_t)p.rows * p.r;
     const __half* opart = reinterpret_cast<const __half*>(p.o_part);
@@ -255,8 +255,8 @@ __global__ void __launch_bounds__(kCombineThreads, 1)
       if (i < nrows) {
         const int bt = row0 + i, b = bt / p.Lq, t = bt % p.Lq, row = t * p.H + h;
         const int sh = c0 / (p.r / S);
-        const int64_t lo = page_owner(p.cum[b], G, p.W) + b;
-        const int64_t hi = page_owner(p.cum[b + 1] - 1, G, p.W) + b;
+        const int64_t lo = page_owner(p.cum[b], b, Gv, p.W) + b;
+        const int64_t hi = page_owner(p.cum[b + 1] - 1, b, Gv, p.W) + b;
         const float* lse = p.lse_part + (int64_t)row * S + sh;
         const __half* op = opart + (int64_t)row * p.r + c0;
         // one round of loads per 4 segments; the running maximum moves as the
