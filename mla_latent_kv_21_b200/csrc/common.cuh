@@ -154,6 +154,10 @@ inline cudaError_t ensure_smem_limit(const void* func, int bytes) {
   for (int i = 0; i < used; ++i)
     if (table[i].func == func && table[i].dev == dev && table[i].bytes >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  // Every kernel of a run asks for the largest shared-memory carveout, so that
+  // consecutive kernels find the SM already configured.
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess && used < 256) table[used++] = Entry{func, dev, bytes};
   return e;
 }

@@ -90,10 +90,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_wuk);
     prefetch_tmap(&tm_qn);
     mbar_arrive_expect_tx_local(bar_w, 8 * 16384);
-    for (int j = 0; j < 8; ++j)  // W_UK[h][:, 64 j .. +64], all 128 d rows
-      tma_load_2d(base + AbsorbSmem::w + 16384 * j, &tm_wuk, 64 * j, h * p.dn, bar_w);
   }
   __syncwarp();
+  // W_UK[h][:, 64 j .. +64], all 128 d rows: one box per lane (a thread's TMA
+  // copies are processed one after another; 8 issuing lanes stream in parallel)
+  if (warp == 0 && lane < 8)
+    tma_load_2d(base + AbsorbSmem::w + 16384 * lane, &tm_wuk, 64 * lane, h * p.dn, bar_w);
   if (warp == 0) {
     tmem_alloc<1>(base + AbsorbSmem::misc, tcols);
     tmem_relinquish<1>();
@@ -222,12 +224,12 @@ __global__ void __launch_bounds__(kCombineThreads, 1)
     // the weights do not depend on the previous kernels: fetch them at once
     prefetch_tmap(&tm_wuv);
     mbar_arrive_expect_tx_local(bar_w, 131072u);
-    for (int j = 0; j < 2; ++j)      // output columns [64 j, 64 j + 64)
-      for (int k = 0; k < 2; ++k)    // latent rows [256 k, 256 k + 256)
-        tma_load_2d(base + CombineSmem::w + 65536 * j + 32768 * k, &tm_wuv, 64 * j, h * p.r + 256 * k,
-                    bar_w);
   }
   __syncwarp();
+  if (warp == 0 && lane < 4) {  // one 32 KB box per lane
+    const int j = lane >> 1, k = lane & 1;  // output columns [64 j, +64), latent rows [256 k, +256)
+    tma_load_2d(base + CombineSmem::w + 65536 * j + 32768 * k, &tm_wuv, 64 * j, h * p.r + 256 * k, bar_w);
+  }
   if (warp == 0) {
     tmem_alloc<1>(base + CombineSmem::misc, 128);
     tmem_relinquish<1>();
