@@ -1,0 +1,72 @@
+"""More parity edge cases of the CUDA path (through the C ABI) against the oracle.
+
+* one 32K-token sequence: every worker of the plan holds a segment of the same
+  sequence, so the combine merges 74 partials per row (many rounds of its
+  four-segment load loop);
+* many short sequences of random lengths, with the default worker count and
+  with 8 workers that each cross several sequence ends (segments of one or
+  two pages, partial groups, query reloads);
+* two plans of different workloads run concurrently on two streams with their
+  own workspaces: results equal the same runs made one after the other.
+"""
+
+import random
+
+import numpy as np
+import pytest
+import torch
+
+import mla_latent_kv_21_b200 as M
+from mla_workloads import WORKLOADS, generate
+
+from harness import assert_close, dims_of, oracle_out, run_gpu, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def test_single_long_sequence_all_workers(cuda_device):
+    wl = WORKLOADS["deepseek_v3"]
+    inputs = generate(wl, seq_lens=[32768])
+    got, info = run_gpu(wl, inputs, cuda_device)
+    assert info.num_workers == 74 and info.num_split_slots == 74
+    got = got.double().numpy()
+    assert np.isfinite(got).all()
+    for h in (0, 77, 127):
+        ref = oracle_out(wl, inputs, [0], [h])[0, :, 0]
+        assert_close(got[0, :, h], ref, wl.dtype, f"h={h}")
+
+
+@pytest.mark.parametrize("workers", [0, 8])
+@pytest.mark.parametrize("name", ["deepseek_v3", "kimi_k2_mtp", "tpla_dsv3"])
+def test_many_short_sequences(cuda_device, name, workers):
+    wl = WORKLOADS[name]
+    rng = random.Random(7)
+    lens = [rng.randint(wl.q_len, 300) for _ in range(40)]
+    inputs = generate(wl, seq_lens=lens)
+    got, info = run_gpu(wl, inputs, cuda_device, num_workers=workers)
+    if workers:
+        assert info.num_workers == workers  # each worker crosses several sequence ends
+    assert_close(got.double().numpy(), oracle_out(wl, inputs), wl.dtype, f"{name} workers={workers}")
+
+
+def test_two_plans_on_two_streams(cuda_device):
+    cases = []
+    for name, lens in (("deepseek_v3", [700, 65, 3000, 1]), ("kimi_k2_mtp", [2, 900, 129, 4000])):
+        wl = WORKLOADS[name]
+        inputs = generate(wl, seq_lens=lens)
+        solo, _ = run_gpu(wl, inputs, cuda_device)
+        dev = to_device(inputs, cuda_device)
+        plan = M.DecodePlan(dims_of(wl), lens).allocate_workspace(cuda_device)
+        out = torch.full((len(lens), wl.q_len, wl.heads, wl.v_dim), float("nan"),
+                         dtype=wl.torch_dtype, device=cuda_device)
+        cases.append((wl, dev, plan, out, solo, torch.cuda.Stream(cuda_device)))
+    torch.cuda.synchronize(cuda_device)
+    for _ in range(3):
+        for wl, dev, plan, out, solo, stream in cases:
+            plan.run(dev["q_nope"], dev["q_rope"], dev["kv_pool"], dev["block_table"],
+                     dev["seq_lens"], dev["w_uk"], dev["w_uv"], out, stream=stream.cuda_stream)
+    torch.cuda.synchronize(cuda_device)
+    for wl, dev, plan, out, solo, stream in cases:
+        assert plan.read_status() == 0
+        assert torch.equal(out.cpu().view(torch.int16), solo.view(torch.int16)), wl.name
+        plan.close()
