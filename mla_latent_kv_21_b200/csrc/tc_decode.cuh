@@ -16,13 +16,15 @@
 //       tensor pipe efficient.
 //   softmax (4 warps per CTA, fp32, log2 domain): per row online max / sum;
 //       the max is moved (and O rescaled) only when it grows by more than 2^8,
-//       so every P value lies in [0, 256] and rescales are rare. Two passes
-//       over the S tile in tensor memory (max, then exp2) keep registers low.
+//       so every P value lies in [0, 256] and rescales are rare. One pass
+//       over the thread's 128 scores in tensor memory (exp2 on the SFU), the
+//       row maximum combined with the other token half through shared memory.
 //   PV  (cta_group::2, M = 128 rows, N = 256 latent columns, K = 256 tokens,
 //       two N blocks): O_lat += P . cKV. CTA c supplies latent columns
 //       [256 nb + 128 c, +128) of every token, streamed page by page through
 //       a second TMA ring (these tokens were just read for QK, so the re-read
-//       is served by L2).
+//       is served by L2). One 16 KB P buffer holds pages 0-1 of the group, then
+//       pages 2-3 once the PV MMAs are done with the first half.
 //   TPLA (S = 2 shards): one S tile per shard (latent chunks 0-3 or 4-7, each
 //       with the RoPE chunk), one softmax per shard, PV N block nb = shard nb.
 //
@@ -32,8 +34,8 @@
 //
 // Each CTA's O accumulator covers its 64 rows x 512 latent columns (256 tensor
 // memory columns). At the end of a split segment the softmax warps write
-// O / l and the log2-sum-exp per row into the workspace; the combine kernel
-// merges the segments and applies W_UV.
+// O / l (fp16) and the log2-sum-exp per row into the workspace; the combine
+// kernel merges the segments and applies W_UV.
 //
 // Sources: TPLA abstract (latent cache, shard-and-sum), TransMLA abstract
 // (absorbed decode over the compressed cache), pith.science verdict record for
