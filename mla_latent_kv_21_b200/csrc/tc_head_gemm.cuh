@@ -46,41 +46,39 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk16) {
 }
 
 // ---------------------------------------------------------------------------
-// absorb: grid (H, ceil(rows / 128)); block 256. One CTA reads all of W_UK[h]
-// (128 KB) once and computes the 4 latent tiles of 128 into 4 tensor-memory
-// accumulators, so 128 heads run as one wave.
-// Shared memory: W_UK[h] [K = 128 d_nope][512 latent] as 8 MN-major groups of
-// 64 latent columns (16 KB each); q_nope rows [N][128] as 2 K-major chunks.
+// absorb: grid (H, 4 latent tiles, ceil(rows / 128)); block 256. One CTA per
+// (head, 128-column latent tile): W_UK[h][:, tile] (32 KB, two MN-major groups
+// of 64 latent columns) as the A operand, q_nope rows [N][128] as 2 K-major
+// chunks; 8 MMAs into one tensor-memory accumulator. Small CTAs (~66 KB of
+// shared memory, 128 registers) so that several share an SM: 4 H CTAs spread
+// the 16.8 MB of W_UK over every SM instead of one 128 KB tile per SM.
 // ---------------------------------------------------------------------------
 constexpr int kAbsorbMaxN = 128;         // query rows per absorb CTA
 struct AbsorbSmem {
-  static constexpr uint32_t w = 0;                             // 128 KB
-  static constexpr uint32_t x = 131072;                        // 2 x N x 128 B <= 32 KB
+  static constexpr uint32_t w = 0;                             // 32 KB
+  static constexpr uint32_t x = 32768;                         // 2 x N x 128 B <= 32 KB
   static constexpr uint32_t bars = x + 2 * kAbsorbMaxN * 128;
   static constexpr uint32_t misc = bars + 64;
   static constexpr uint32_t alloc = misc + 64 + 1024;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_wuk,
                      const __grid_constant__ CUtensorMap tm_qn, RunParams p, int n_pad) {
   using namespace ptx;
   extern __shared__ uint8_t smem_raw[];
-  // page prefix sums and length check of this run (all 256 threads of one block)
   if (threadIdx.x == 0) MLA_HG_TRACE(0, 0);
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const int h = blockIdx.x;
+  const int h = blockIdx.x, mt = blockIdx.y;  // head, latent tile [128 mt, +128)
   const int nbt = p.B * p.Lq;
-  const int row0 = blockIdx.y * kAbsorbMaxN;
+  const int row0 = blockIdx.z * kAbsorbMaxN;
   const int nrows = min(kAbsorbMaxN, nbt - row0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t bar_w = base + AbsorbSmem::bars, bar_x = bar_w + 8, bar_done = bar_w + 16;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(gbase + AbsorbSmem::misc);
-  // tensor memory: 4 accumulators of n_pad columns (n_pad <= 128)
-  const uint32_t tcols = 4 * n_pad <= 32 ? 32 : 4 * n_pad <= 64 ? 64 : 4 * n_pad <= 128 ? 128 :
-                         4 * n_pad <= 256 ? 256 : 512;
+  const uint32_t tcols = n_pad <= 32 ? 32 : n_pad <= 64 ? 64 : 128;
   if (threadIdx.x == 0) {
     mbar_init(bar_w, 1);
     mbar_init(bar_x, 1);
@@ -89,13 +87,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the weights do not depend on the previous kernel: fetch them at once
     prefetch_tmap(&tm_wuk);
     prefetch_tmap(&tm_qn);
-    mbar_arrive_expect_tx_local(bar_w, 8 * 16384);
+    mbar_arrive_expect_tx_local(bar_w, 2 * 16384);
   }
   __syncwarp();
-  // W_UK[h][:, 64 j .. +64], all 128 d rows: one box per lane (a thread's TMA
-  // copies are processed one after another; 8 issuing lanes stream in parallel)
-  if (warp == 0 && lane < 8)
-    tma_load_2d(base + AbsorbSmem::w + 16384 * lane, &tm_wuk, 64 * lane, h * p.dn, bar_w);
+  // W_UK[h][:, 128 mt + 64 j .. +64], all 128 d rows: one box per lane
+  if (warp == 0 && lane < 2)
+    tma_load_2d(base + AbsorbSmem::w + 16384 * lane, &tm_wuk, 128 * mt + 64 * lane, h * p.dn, bar_w);
   if (warp == 0) {
     tmem_alloc<1>(base + AbsorbSmem::misc, tcols);
     tmem_relinquish<1>();
@@ -109,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   grid_launch_dependents();
   grid_dependency_wait();
   // page prefix sums and length check of this run (all 256 threads of one block)
-  if (blockIdx.x == 0 && blockIdx.y == 0) scan_lengths(p);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) scan_lengths(p);
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx_local(bar_x, 2 * n_pad * 128);
     for (int kc = 0; kc < 2; ++kc)  // q_nope rows [row0, row0 + n_pad), d chunk kc
@@ -119,21 +116,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(128, n_pad, 1, 0);
       const uint64_t b0 = smem_desc_sw128(base + AbsorbSmem::x, 16, 1024);
-      for (int mt = 0; mt < 4; ++mt) {  // latent tile [128 mt, +128): groups 2 mt, 2 mt + 1
-        const uint64_t a0 = smem_desc_sw128(base + AbsorbSmem::w + 32768 * mt, 16384, 1024);
-        for (int ks = 0; ks < 8; ++ks) {  // K = 128 = 8 x 16
-          const uint64_t ad = a0 + (uint64_t)(128 * ks);  // 16 K rows x 128 B
-          const uint64_t bd = b0 + (uint64_t)(((ks >> 2) * n_pad * 128) >> 4) + (uint64_t)(2 * (ks & 3));
-          mma_f16<1>(tbase + mt * n_pad, ad, bd, idesc, ks > 0 ? 1u : 0u);
-        }
+      const uint64_t a0 = smem_desc_sw128(base + AbsorbSmem::w, 16384, 1024);
+      for (int ks = 0; ks < 8; ++ks) {  // K = 128 = 8 x 16
+        const uint64_t ad = a0 + (uint64_t)(128 * ks);  // 16 K rows x 128 B
+        const uint64_t bd = b0 + (uint64_t)(((ks >> 2) * n_pad * 128) >> 4) + (uint64_t)(2 * (ks & 3));
+        mma_f16<1>(tbase, ad, bd, idesc, ks > 0 ? 1u : 0u);
       }
       tc_commit<1>(bar_done);
     } else {
       record_error(p.status, MLA_ERR_DEVICE_TIMEOUT);
     }
   }
-  // q_rope columns of the packed query rows
-  {
+  // q_rope columns of the packed query rows (the tile-0 CTA of each head)
+  if (mt == 0) {
     const __nv_bfloat16* q_rope = static_cast<const __nv_bfloat16*>(p.q_rope);
     __nv_bfloat16* q = static_cast<__nv_bfloat16*>(p.q);
     for (int idx = threadIdx.x; idx < nrows * p.dr; idx += blockDim.x) {
@@ -143,25 +138,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncwarp();
   {
-    // warps w and w + 4 share lane quadrant w % 4: tiles {0, 1} and {2, 3}
+    // warps w and w + 4 share lane quadrant w % 4 (latent columns
+    // 32 (w % 4) .. +32 of the tile) and split the rows by 32-row chunks
     const bool done = mbar_wait(bar_done, 0);
     if (threadIdx.x == 0) MLA_HG_TRACE(0, 2);
     if (__all_sync(0xffffffffu, done)) {
       tc_fence_after();
       __nv_bfloat16* q = static_cast<__nv_bfloat16*>(p.q);
       const int quad = warp & 3;
-      const int m = 32 * quad + lane;  // latent column within a tile
-      for (int mt = 2 * (warp >> 2); mt < 2 * (warp >> 2) + 2; ++mt) {
-        for (int c0 = 0; c0 < n_pad; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(tbase + ((uint32_t)(32 * quad) << 16) + mt * n_pad + c0, r);
-          tmem_wait_ld();
-          for (int j = 0; j < 32; ++j) {
-            const int i = c0 + j;
-            if (i < nrows)
-              q[((int64_t)(row0 + i) * p.H + h) * (p.r + p.dr) + 128 * mt + m] =
-                  __float2bfloat16_rn(__uint_as_float(r[j]));
-          }
+      const int m = 128 * mt + 32 * quad + lane;  // latent column
+      for (int c0 = 32 * (warp >> 2); c0 < n_pad; c0 += 64) {
+        uint32_t r[32];
+        tmem_ld32(tbase + ((uint32_t)(32 * quad) << 16) + c0, r);
+        tmem_wait_ld();
+        for (int j = 0; j < 32; ++j) {
+          const int i = c0 + j;
+          if (i < nrows)
+            q[((int64_t)(row0 + i) * p.H + h) * (p.r + p.dr) + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
         }
       }
     } else if (lane == 0) {
@@ -402,7 +395,7 @@ inline cudaError_t launch_absorb_tc(const RunParams& p, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(hg::absorb_tc_kernel), (int)hg::AbsorbSmem::alloc);
   if (e != cudaSuccess) return e;
-  const dim3 grid(p.H, (nbt + hg::kAbsorbMaxN - 1) / hg::kAbsorbMaxN);
+  const dim3 grid(p.H, 4, (nbt + hg::kAbsorbMaxN - 1) / hg::kAbsorbMaxN);  // r = 512: 4 latent tiles
   return launch_dependent(hg::absorb_tc_kernel, grid, dim3(hg::kThreads), hg::AbsorbSmem::alloc,
                               stream, tm_wuk, tm_qn, p, n_pad);
 }
