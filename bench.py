@@ -64,7 +64,10 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------------------
-# algorithmic work of one step (measurement)
+# algorithmic work of one step: cache bytes (r + d_rope elements per cached
+# token), absorbed-query bytes (one query row per sequence and head), weight and
+# output bytes, and the FLOPs of the absorb, QK, PV and up-projection
+# contractions
 # ----------------------------------------------------------------------------
 def step_work(wl, lens):
     elt = 2 if wl.dtype == "bf16" else 4
