@@ -160,3 +160,34 @@ def test_workspace_holds_partials_for_every_slot():
         assert ws >= need
     finally:
         L.mla_plan_destroy(plan)
+
+
+@pytest.mark.parametrize("kw,kernel,status", [
+    # the latent-split kernel takes one latent shard, bf16
+    (dict(latent_shards=2), L.MLA_KERNEL_TCGEN05_LSPLIT, L.MLA_ERR_UNSUPPORTED),
+    # the tensor-core kernels need r = 512 bf16; the fp32 tiny shape is SIMT only
+    (dict(latent_rank=64, rope_dim=16, nope_dim=32, v_dim=32, dtype="fp32"),
+     L.MLA_KERNEL_TCGEN05, L.MLA_ERR_UNSUPPORTED),
+    (dict(latent_rank=64, rope_dim=16, nope_dim=32, v_dim=32, dtype="fp32"),
+     L.MLA_KERNEL_TCGEN05_LSPLIT, L.MLA_ERR_UNSUPPORTED),
+    # unknown kernel kind
+    (dict(), 7, L.MLA_ERR_INVALID_ARG),
+])
+def test_plan_rejects_unsupported_kernel_choices(kw, kernel, status):
+    with pytest.raises(L.MlaError) as e:
+        L.mla_decode_plan_ex(_dims(**kw), [100, 200], num_sms=148, kernel=kernel)
+    assert e.value.status == status
+
+
+@pytest.mark.parametrize("kernel", [L.MLA_KERNEL_AUTO, L.MLA_KERNEL_TCGEN05, L.MLA_KERNEL_TCGEN05_LSPLIT,
+                                    L.MLA_KERNEL_SIMT])
+def test_plan_reports_kernel_and_launches(kernel):
+    plan, ws = L.mla_decode_plan_ex(_dims(), [4000, 65], num_sms=148, kernel=kernel)
+    try:
+        info = L.mla_plan_get_info(plan)
+        want = L.MLA_KERNEL_TCGEN05 if kernel == L.MLA_KERNEL_AUTO else kernel
+        assert info.kernel == want
+        assert info.launches_per_run == 3
+        assert info.workspace_bytes == ws > 0
+    finally:
+        L.mla_plan_destroy(plan)
