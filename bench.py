@@ -70,12 +70,13 @@ def load_peaks():
 # contractions
 # ----------------------------------------------------------------------------
 def step_work(wl, lens):
-    elt = 2 if wl.dtype == "bf16" else 4
+    elt = 4 if wl.dtype == "fp32" else 2
     B, Lq, H = len(lens), wl.q_len, wl.heads
     r, dr, dn, dv, S = wl.latent_rank, wl.rope_dim, wl.nope_dim, wl.v_dim, wl.latent_shards
     sum_l = int(sum(lens))
     rows = H * Lq
-    cache = sum_l * (r + dr) * elt
+    # FP8 cache: r code bytes, the bf16 RoPE key and an fp32 scale per token
+    cache = sum_l * (r + dr * 2 + 4) if wl.dtype == "fp8" else sum_l * (r + dr) * elt
     q_full = B * rows * (r + dr) * elt
     weights = H * dn * r * elt + H * r * dv * elt
     io = B * rows * (dn + dr) * elt + B * rows * dv * elt
@@ -304,8 +305,8 @@ def time_oracle_sample(wl, inputs, pairs, tokens):
     """Runs the oracle on (sequence, head) pairs over their first `tokens` keys
     (Lq = 1 workloads) or full length; returns (seconds, outputs)."""
     import numpy as np
-    from mla_workloads import logical_cache
-    from oracle import mla_oracle
+    from mla_workloads import logical_cache, stored_rows_fp8
+    from oracle import fp8_cache, mla_oracle
     qn = inputs["q_nope"].double().numpy()
     qr = inputs["q_rope"].double().numpy()
     wuk = inputs["w_uk"].double().numpy()
@@ -313,10 +314,14 @@ def time_oracle_sample(wl, inputs, pairs, tokens):
     outs = []
     t0 = time.perf_counter()
     for b, h in pairs:
-        c, k = logical_cache(inputs, b, wl)
+        if wl.dtype == "fp8":
+            codes, rope, scale = stored_rows_fp8(inputs, b, wl)
+            c, k = fp8_cache.logical_cache_fp8(codes.numpy(), rope.double().numpy(), scale.double().numpy())
+        else:
+            c, k = logical_cache(inputs, b, wl)
+            c, k = c.double().numpy(), k.double().numpy()
         n = min(tokens, c.shape[0]) if tokens else c.shape[0]
-        outs.append(mla_oracle.mla_decode(qn, qr, {b: c[:n].double().numpy()},
-                                          {b: k[:n].double().numpy()}, wuk, wuv,
+        outs.append(mla_oracle.mla_decode(qn, qr, {b: c[:n]}, {b: k[:n]}, wuk, wuv,
                                           wl.softmax_scale, wl.latent_shards, [b], [h]))
     return time.perf_counter() - t0, outs
 
@@ -330,8 +335,8 @@ def compare_sample(gpu_out, oracle_outs, pairs, dtype):
     return {"max_abs": float(np.abs(d).max()),
             "rel_fro": float(np.linalg.norm(d) / np.linalg.norm(ref)),
             "pairs": [list(p) for p in pairs],
-            "tolerance": ({"max_abs": 2e-2, "rel_fro": 5e-3} if dtype == "bf16"
-                          else {"rel_fro": 1e-5})}
+            "tolerance": ({"rel_fro": 1e-5} if dtype == "fp32"
+                          else {"max_abs": 2e-2, "rel_fro": 5e-3})}
 
 
 def reference_arm(args, wl, world, rank):
@@ -414,9 +419,16 @@ def main():
     out = torch.empty((B, wl.q_len, wl.heads, wl.v_dim), dtype=wl.torch_dtype, device=device)
     stream = torch.cuda.current_stream(device)
 
+    def run_plan(q_nope, q_rope, block_table, seq_lens, o, events=None):
+        if wl.dtype == "fp8":
+            plan.run_fp8(q_nope, q_rope, dev["kv_codes"], dev["kv_rope"], dev["kv_scale"], block_table,
+                         seq_lens, dev["w_uk"], dev["w_uv"], o, stream.cuda_stream, events)
+        else:
+            plan.run(q_nope, q_rope, dev["kv_pool"], block_table, seq_lens, dev["w_uk"], dev["w_uv"], o,
+                     stream.cuda_stream, events)
+
     def step(events=None):
-        plan.run(dev["q_nope"], dev["q_rope"], dev["kv_pool"], dev["block_table"],
-                 dev["seq_lens"], dev["w_uk"], dev["w_uv"], out, stream.cuda_stream, events)
+        run_plan(dev["q_nope"], dev["q_rope"], dev["block_table"], dev["seq_lens"], out, events)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -490,8 +502,7 @@ def main():
             if i >= 2:
                 stream.wait_event(ev["d2h"][b])        # out b of step i-2 has been copied out
             d = dsets[b]
-            plan.run(d["q_nope"], d["q_rope"], dev["kv_pool"], d["block_table"], d["seq_lens"],
-                     dev["w_uk"], dev["w_uv"], douts[b], stream.cuda_stream)
+            run_plan(d["q_nope"], d["q_rope"], d["block_table"], d["seq_lens"], douts[b])
             ev["comp"][b].record(stream)
             d2h_stream.wait_event(ev["comp"][b])
             with torch.cuda.stream(d2h_stream):
@@ -524,7 +535,12 @@ def main():
         info.kernel, "simt")
     dec_s = statistics.mean(decode_ms) * 1e-3
     hbm_peak = peaks["hbm_gbs"]
-    if kname.startswith("tcgen05"):
+    if kname.startswith("tcgen05") and wl.dtype == "fp8":
+        # e4m3 / e5m2 MMAs: the fp8 dense rate is twice bf16's (nominal ratio);
+        # the two-term operand splits execute 2x the algorithmic FLOPs there
+        flop_peak = 2 * peaks["bf16_tflops"]
+        flop_kind = "fp8 tensor = 2 x measured bf16"
+    elif kname.startswith("tcgen05"):
         flop_peak = peaks["bf16_tflops"]
         flop_kind = "bf16 tensor"
     else:
@@ -546,8 +562,10 @@ def main():
     roof["peak_source"] = f"{peaks_kind} ({flop_kind} for FLOPs)"
     roof["decode_us"] = dec_s * 1e6
     roof["decode_launches_timed"] = Kd
+    fp8_dec = work["decode_flops"] if wl.dtype == "fp8" else 0
     step_roof_s = max(work["step_bytes"] / (hbm_peak * 1e9),
-                      work["step_flops"] / (peaks["bf16_tflops"] * 1e12))
+                      (work["step_flops"] - fp8_dec) / (peaks["bf16_tflops"] * 1e12)
+                      + fp8_dec / (2 * peaks["bf16_tflops"] * 1e12))
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,

@@ -67,7 +67,10 @@ typedef enum {
   MLA_ERR_NO_DEVICE = 7            /* no usable sm_100 device */
 } mla_status_t;
 
-typedef enum { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype_t;
+/* MLA_FP8_CACHE: activations, weights and output bf16; the cache holds per
+ * token r E4M3 codes of cKV, one fp32 scale s_t and the RoPE key in bf16
+ * divided by s_t (see mla_decode_run_fp8). Tensor-core path, one latent shard. */
+typedef enum { MLA_BF16 = 0, MLA_FP32 = 1, MLA_FP8_CACHE = 2 } mla_dtype_t;
 
 /* Kernel family selection (mla_plan_options_t.kernel). */
 typedef enum {
@@ -159,6 +162,29 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan,
                                const void* w_uk, const void* w_uv,
                                void* out, void* workspace, size_t workspace_bytes,
                                void* stream, const mla_run_options_t* opts);
+
+/* One decode step over an FP8 latent cache (plan made with dims.dtype =
+ * MLA_FP8_CACHE; mla_decode_run / _ex refuse such a plan with
+ * MLA_ERR_INVALID_ARG). The cache is three device tensors over the same
+ * blocks:
+ *   kv_codes uint8 [num_blocks, page_size, r]   E4M3 ("e4m3fn") codes of cKV
+ *   kv_rope  bf16  [num_blocks, page_size, d_rope] RoPE key divided by s_t
+ *   kv_scale fp32  [num_blocks, page_size]      s_t, so that cKV_t = s_t * code_t
+ *                                               and k_rope_t = s_t * kv_rope_t
+ * (kv_scale 16-byte aligned). Every other argument, the workspace and the
+ * errors are as for mla_decode_run_ex. The tensor-core MMAs take e4m3 / e5m2
+ * operands: the absorbed query and P * s_t each as an e4m3 value plus an e5m2
+ * correction, so that the result stays within the bf16 tolerance of the
+ * dequantised cache; P * s_t must stay below 448 (s_t <= 1.75). */
+mla_status_t mla_decode_run_fp8(mla_plan_t plan,
+                                const void* q_nope, const void* q_rope,
+                                const void* kv_codes, const void* kv_rope, const float* kv_scale,
+                                int64_t num_blocks,
+                                const int32_t* block_table, int32_t block_table_stride,
+                                const int32_t* seq_lens_dev,
+                                const void* w_uk, const void* w_uv,
+                                void* out, void* workspace, size_t workspace_bytes,
+                                void* stream, const mla_run_options_t* opts);
 
 /* Decode step without a caller workspace, for callers that cannot allocate
  * device memory where they run decode steps (an engine whose memory pool owns

@@ -34,6 +34,7 @@ MLA_ERR_NO_DEVICE = 7
 
 MLA_BF16 = 0
 MLA_FP32 = 1
+MLA_FP8_CACHE = 2
 
 MLA_KERNEL_AUTO = 0
 MLA_KERNEL_SIMT = 1
@@ -43,7 +44,7 @@ MLA_KERNEL_TCGEN05_LSPLIT = 3
 # symbols declared in include/mla_decode.h
 EXPORTED = (
     "mla_decode_plan", "mla_decode_plan_ex", "mla_decode_run", "mla_decode_run_ex",
-    "mla_decode_run_no_alloc", "mla_workspace_init",
+    "mla_decode_run_fp8", "mla_decode_run_no_alloc", "mla_workspace_init",
     "mla_decode_read_status", "mla_plan_get_info", "mla_plan_segments", "mla_plan_destroy",
     "mla_status_string", "mla_abi_version",
 )
@@ -93,6 +94,9 @@ _lib.mla_decode_run.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _
 _lib.mla_decode_run_ex.restype = ctypes.c_int
 _lib.mla_decode_run_ex.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
                                    _sz, _vp, ctypes.POINTER(mla_run_options_t)]
+_lib.mla_decode_run_fp8.restype = ctypes.c_int
+_lib.mla_decode_run_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp,
+                                    _vp, _sz, _vp, ctypes.POINTER(mla_run_options_t)]
 _lib.mla_decode_run_no_alloc.restype = ctypes.c_int
 _lib.mla_decode_run_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp,
                                          _vp]
@@ -174,6 +178,18 @@ def mla_decode_run_ex(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,
                                   block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace,
                                   workspace_bytes, stream, ctypes.byref(opts)),
            "mla_decode_run_ex")
+
+
+def mla_decode_run_fp8(plan, q_nope, q_rope, kv_codes, kv_rope, kv_scale, num_blocks, block_table,
+                       block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace,
+                       workspace_bytes, stream=0, decode_start_event=None,
+                       decode_stop_event=None) -> None:
+    """One decode step over an FP8 latent cache (codes, RoPE key / scale, scales)."""
+    opts = mla_run_options_t(decode_start_event, decode_stop_event)
+    _check(_lib.mla_decode_run_fp8(plan, q_nope, q_rope, kv_codes, kv_rope, kv_scale, num_blocks,
+                                   block_table, block_table_stride, seq_lens_dev, w_uk, w_uv, out,
+                                   workspace, workspace_bytes, stream, ctypes.byref(opts)),
+           "mla_decode_run_fp8")
 
 
 def mla_decode_run_no_alloc(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,

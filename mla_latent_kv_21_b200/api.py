@@ -11,9 +11,9 @@ from . import _lib as L
 def dims_for(heads: int, latent_rank: int, rope_dim: int, nope_dim: int, v_dim: int,
              q_len: int, softmax_scale: float, dtype: str = "bf16", latent_shards: int = 1,
              page_size: int = 64) -> L.mla_dims_t:
+    code = {"bf16": L.MLA_BF16, "fp32": L.MLA_FP32, "fp8": L.MLA_FP8_CACHE}[dtype]
     return L.make_dims(heads, latent_rank, rope_dim, nope_dim, v_dim, q_len, page_size,
-                       latent_shards, float(softmax_scale),
-                       L.MLA_BF16 if dtype == "bf16" else L.MLA_FP32)
+                       latent_shards, float(softmax_scale), code)
 
 
 class DecodePlan:
@@ -57,6 +57,26 @@ class DecodePlan:
                             block_table.shape[1], seq_lens.data_ptr(), w_uk.data_ptr(),
                             w_uv.data_ptr(), out.data_ptr(), self.workspace.data_ptr(),
                             self.workspace_bytes, stream, ev0, ev1)
+
+    def run_fp8(self, q_nope, q_rope, kv_codes, kv_rope, kv_scale, block_table, seq_lens, w_uk,
+                w_uv, out, stream: Optional[int] = None, decode_events=None) -> None:
+        """As run, over an FP8 latent cache (include/mla_decode.h, mla_decode_run_fp8)."""
+        import torch
+        if self.workspace is None:
+            self.allocate_workspace(q_nope.device)
+        for name, t in (("q_nope", q_nope), ("q_rope", q_rope), ("kv_codes", kv_codes),
+                        ("kv_rope", kv_rope), ("kv_scale", kv_scale), ("block_table", block_table),
+                        ("seq_lens", seq_lens), ("w_uk", w_uk), ("w_uv", w_uv), ("out", out)):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if stream is None:
+            stream = torch.cuda.current_stream(q_nope.device).cuda_stream
+        ev0, ev1 = (None, None) if decode_events is None else decode_events
+        L.mla_decode_run_fp8(self.handle, q_nope.data_ptr(), q_rope.data_ptr(), kv_codes.data_ptr(),
+                             kv_rope.data_ptr(), kv_scale.data_ptr(), kv_codes.shape[0],
+                             block_table.data_ptr(), block_table.shape[1], seq_lens.data_ptr(),
+                             w_uk.data_ptr(), w_uv.data_ptr(), out.data_ptr(),
+                             self.workspace.data_ptr(), self.workspace_bytes, stream, ev0, ev1)
 
     def read_status(self, stream: Optional[int] = None) -> int:
         import torch

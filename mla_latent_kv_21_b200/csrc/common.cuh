@@ -105,7 +105,9 @@ struct RunParams {
   // inputs
   const void* q_nope;
   const void* q_rope;
-  const void* kv;          // pool
+  const void* kv;          // pool (bf16 / fp32 rows, or the e4m3 codes of an FP8 cache)
+  const void* kv_rope;     // FP8 cache: bf16 RoPE keys stored divided by the token scale
+  const float* kv_scale;   // FP8 cache: fp32 scale per token [num_blocks, page_size]
   const int32_t* block_table;
   const int32_t* seq_lens;
   const void* w_uk;
@@ -124,6 +126,7 @@ struct RunParams {
   int32_t B, Lq, H, r, dr, dn, dv, P, S;
   int32_t rows;            // H * Lq
   int32_t W;               // workers
+  int32_t fp8;             // 1: FP8 cache (the absorbed query is written as e4m3 + e5m2 bytes)
   float scale_log2;        // softmax_scale * log2(e)
 };
 

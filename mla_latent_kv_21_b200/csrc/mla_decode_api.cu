@@ -12,6 +12,7 @@
 #include "simt_kernels.cuh"
 #include "tc_decode.cuh"
 #include "tc_decode_ls.cuh"
+#include "tc_decode_f8.cuh"
 #include "tc_head_gemm.cuh"
 
 using namespace mla;
@@ -30,9 +31,9 @@ struct mla_plan {
 namespace {
 
 bool tc_supported(const mla_dims_t& d) {
-  return kTcDecodeAvailable && d.dtype == MLA_BF16 && d.latent_rank == 512 && d.rope_dim == 64 && d.page_size == 64 &&
-         d.num_heads * d.q_len <= 128 && d.nope_dim == 128 && d.v_dim == 128 &&
-         (d.latent_shards == 1 || d.latent_shards == 2);
+  return kTcDecodeAvailable && (d.dtype == MLA_BF16 || d.dtype == MLA_FP8_CACHE) && d.latent_rank == 512 &&
+         d.rope_dim == 64 && d.page_size == 64 && d.num_heads * d.q_len <= 128 && d.nope_dim == 128 &&
+         d.v_dim == 128 && (d.latent_shards == 1 || (d.latent_shards == 2 && d.dtype == MLA_BF16));
 }
 
 mla_status_t check_dims(const mla_dims_t& d) {
@@ -40,7 +41,7 @@ mla_status_t check_dims(const mla_dims_t& d) {
       d.q_len < 1 || d.page_size < 1 || d.latent_shards < 1 || !std::isfinite(d.softmax_scale) ||
       d.softmax_scale <= 0.f)
     return MLA_ERR_INVALID_ARG;
-  if (d.dtype != MLA_BF16 && d.dtype != MLA_FP32) return MLA_ERR_INVALID_ARG;
+  if (d.dtype != MLA_BF16 && d.dtype != MLA_FP32 && d.dtype != MLA_FP8_CACHE) return MLA_ERR_INVALID_ARG;
   if (d.page_size != 64) return MLA_ERR_UNSUPPORTED;
   if (d.latent_shards > 2 || d.latent_rank % d.latent_shards != 0) return MLA_ERR_UNSUPPORTED;
   if (d.latent_rank > 512 || d.latent_rank + d.rope_dim > 576 || d.nope_dim > kMaxNope ||
@@ -97,6 +98,9 @@ mla_status_t mla_decode_plan_ex(const mla_dims_t* dims, int32_t batch, const int
   }
   int32_t kernel = o.kernel;
   if (kernel == MLA_KERNEL_AUTO) kernel = tc_supported(*dims) ? MLA_KERNEL_TCGEN05 : MLA_KERNEL_SIMT;
+  // the FP8 cache has one kernel: tcgen05, one latent shard
+  if (dims->dtype == MLA_FP8_CACHE && (kernel != MLA_KERNEL_TCGEN05 || !tc_supported(*dims)))
+    return MLA_ERR_UNSUPPORTED;
   if (kernel == MLA_KERNEL_TCGEN05 && !tc_supported(*dims)) return MLA_ERR_UNSUPPORTED;
   if (kernel == MLA_KERNEL_TCGEN05_LSPLIT && !(tc_supported(*dims) && dims->latent_shards == 1))
     return MLA_ERR_UNSUPPORTED;
@@ -121,7 +125,7 @@ mla_status_t mla_decode_plan_ex(const mla_dims_t* dims, int32_t batch, const int
   p->num_sms = sms;
   p->G = G;
   p->lens.assign(seq_lens_host, seq_lens_host + batch);
-  const int elt = dims->dtype == MLA_BF16 ? 2 : 4;
+  const int elt = dims->dtype == MLA_FP32 ? 4 : 2;  // FP8 cache: query rows of 2 (r + d_rope) bytes
   p->layout = workspace_layout(batch, dims->q_len, dims->num_heads, dims->latent_rank,
                                dims->rope_dim, dims->latent_shards, elt, W + batch - 1);
   *plan_out = p;
@@ -190,12 +194,15 @@ mla_status_t mla_decode_run(mla_plan_t plan, const void* q_nope, const void* q_r
                            workspace_bytes, stream_, nullptr);
 }
 
-mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* q_rope,
-                               const void* kv_cache, int64_t num_blocks,
-                               const int32_t* block_table, int32_t block_table_stride,
-                               const int32_t* seq_lens_dev, const void* w_uk, const void* w_uv,
-                               void* out, void* workspace, size_t workspace_bytes, void* stream_,
-                               const mla_run_options_t* opts) {
+}  // extern "C"
+
+namespace {
+
+mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, const void* kv_cache,
+                      const void* kv_rope, const float* kv_scale, int64_t num_blocks,
+                      const int32_t* block_table, int32_t block_table_stride, const int32_t* seq_lens_dev,
+                      const void* w_uk, const void* w_uv, void* out, void* workspace, size_t workspace_bytes,
+                      void* stream_, const mla_run_options_t* opts) {
   if (!plan || !q_nope || !q_rope || !kv_cache || !block_table || !seq_lens_dev || !w_uk ||
       !w_uv || !out || !workspace || num_blocks < 1 || block_table_stride < 1)
     return MLA_ERR_INVALID_ARG;
@@ -208,6 +215,9 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* 
   p.q_nope = q_nope;
   p.q_rope = q_rope;
   p.kv = kv_cache;
+  p.kv_rope = kv_rope;
+  p.kv_scale = kv_scale;
+  p.fp8 = plan->dims.dtype == MLA_FP8_CACHE ? 1 : 0;
   p.block_table = block_table;
   p.seq_lens = seq_lens_dev;
   p.w_uk = w_uk;
@@ -249,7 +259,9 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* 
   cudaEvent_t ev_start = opts ? static_cast<cudaEvent_t>(opts->decode_start_event) : nullptr;
   cudaEvent_t ev_stop = opts ? static_cast<cudaEvent_t>(opts->decode_stop_event) : nullptr;
   if (ev_start && cudaEventRecord(ev_start, stream) != cudaSuccess) return MLA_ERR_CUDA;
-  if (plan->kernel == MLA_KERNEL_TCGEN05) {
+  if (p.fp8) {
+    if (launch_tc_decode_f8(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
+  } else if (plan->kernel == MLA_KERNEL_TCGEN05) {
     if (launch_tc_decode(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
   } else if (plan->kernel == MLA_KERNEL_TCGEN05_LSPLIT) {
     if (launch_ls_decode(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
@@ -281,6 +293,32 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* 
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status_t mla_decode_run_ex(mla_plan_t plan, const void* q_nope, const void* q_rope,
+                               const void* kv_cache, int64_t num_blocks,
+                               const int32_t* block_table, int32_t block_table_stride,
+                               const int32_t* seq_lens_dev, const void* w_uk, const void* w_uv,
+                               void* out, void* workspace, size_t workspace_bytes, void* stream_,
+                               const mla_run_options_t* opts) {
+  if (plan && plan->dims.dtype == MLA_FP8_CACHE) return MLA_ERR_INVALID_ARG;  // mla_decode_run_fp8
+  return run_impl(plan, q_nope, q_rope, kv_cache, nullptr, nullptr, num_blocks, block_table,
+                  block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace, workspace_bytes, stream_, opts);
+}
+
+mla_status_t mla_decode_run_fp8(mla_plan_t plan, const void* q_nope, const void* q_rope,
+                                const void* kv_codes, const void* kv_rope, const float* kv_scale,
+                                int64_t num_blocks, const int32_t* block_table,
+                                int32_t block_table_stride, const int32_t* seq_lens_dev,
+                                const void* w_uk, const void* w_uv, void* out, void* workspace,
+                                size_t workspace_bytes, void* stream_, const mla_run_options_t* opts) {
+  if (!plan || plan->dims.dtype != MLA_FP8_CACHE || !kv_rope || !kv_scale) return MLA_ERR_INVALID_ARG;
+  return run_impl(plan, q_nope, q_rope, kv_codes, kv_rope, kv_scale, num_blocks, block_table,
+                  block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace, workspace_bytes, stream_, opts);
 }
 
 mla_status_t mla_workspace_init(void* workspace, size_t workspace_bytes, void* stream_) {

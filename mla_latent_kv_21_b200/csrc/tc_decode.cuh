@@ -167,7 +167,7 @@ __device__ unsigned long long g_trace_chunk[4 * kTraceChunks];
 #define MLA_TRACE_CTA(k) do {} while (0)
 #endif
 enum { EV_QK_START = 0, EV_QK_END, EV_PV_START, EV_PV_END, EV_S_READY, EV_P_DONE, EV_PBUF_FREE, EV_LOAD,
-       EV_PASS1, EV_PASS2, EV_SYNC1, EV_LD0 };
+       EV_PASS1, EV_PASS2, EV_SYNC1, EV_LD0, EV_LD1, EV_LD2, EV_LD3 };
 
 // Sequential walk over a worker's page groups: sequence b, first page and
 // page count of the group (1..4), first-group-of-segment flag, segment index.

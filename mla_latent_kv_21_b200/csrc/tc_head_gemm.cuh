@@ -153,8 +153,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_wait_ld();
         for (int j = 0; j < 32; ++j) {
           const int i = c0 + j;
-          if (i < nrows)
-            q[((int64_t)(row0 + i) * p.H + h) * (p.r + p.dr) + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
+          if (i >= nrows) continue;
+          const int64_t qrow = (int64_t)(row0 + i) * p.H + h;
+          const float v = __uint_as_float(r[j]);
+          if (p.fp8) {
+            // FP8 cache: the query row is [e4m3(q) x r | e5m2(q - e4m3(q)) x r |
+            // bf16 q_rope], 2 (r + d_rope) bytes like the bf16 row
+            uint8_t* qb = static_cast<uint8_t*>(p.q) + qrow * 2 * (p.r + p.dr);
+            const uint32_t hi = cvt_e4m3x2(v, 0.f);
+            const float back = e4m3x2_to_float2(hi).x;
+            qb[m] = (uint8_t)(hi & 0xFF);
+            qb[p.r + m] = (uint8_t)(cvt_e5m2x2(v - back, 0.f) & 0xFF);
+          } else {
+            q[qrow * (p.r + p.dr) + m] = __float2bfloat16_rn(v);
+          }
         }
       }
     } else if (lane == 0) {

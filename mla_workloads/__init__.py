@@ -18,6 +18,10 @@ synthetic because no trained weights are available):
                   [1024, 32768], 2 causal query tokens per sequence, paged
 * ``tpla_dsv3``   bf16, DeepSeek-V3 shape with the latent split into 2 shards
                   (TPLA), B=32, L=32768, paged
+* ``deepseek_v3_fp8`` the DeepSeek-V3 shape over an FP8 latent cache: cKV as
+                  E4M3 codes with one fp32 scale per token, the RoPE key bf16
+                  stored divided by the token's scale; activations and weights
+                  bf16
 
 Recipe (every draw is float32 N(0, 1) from ``torch.Generator`` seeded per
 tensor, then scaled and cast to the workload dtype with round-to-nearest-even):
@@ -35,6 +39,14 @@ tensor, then scaled and cast to the workload dtype with round-to-nearest-even):
   place logical page (b, i) at a block chosen by a seeded random permutation,
   contiguous ones at the identity position. Unused table entries are -1 and
   the tail of a partial page is zero.
+
+FP8 cache (``dtype="fp8"``): the same per-sequence N(0, 1) block, times 32, is
+cast to E4M3 codes with torch's own conversion (columns [0, r)) and to bf16
+(columns [r, r + dr), the stored RoPE key); each token's scale is uniform in
+[1/48, 1/24] (tag ``200 + b``). The logical cache is s_t * code and
+s_t * stored RoPE key; the CPU oracle decodes it (``oracle/fp8_cache.py``).
+The pool is three tensors: kv_codes uint8 [blocks, P, r], kv_rope bf16
+[blocks, P, dr] and kv_scale float32 [blocks, P] (zero in unused slots).
 """
 
 from __future__ import annotations
@@ -45,7 +57,7 @@ from typing import Optional, Sequence
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "generate", "logical_cache", "pages_of"]
+__all__ = ["Workload", "WORKLOADS", "generate", "logical_cache", "pages_of", "stored_rows_fp8"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -62,7 +74,7 @@ class Workload:
     context: int            # fixed length, or the upper bound when varlen
     context_min: int = 0    # > 0 selects uniform integer lengths in [context_min, context]
     latent_shards: int = 1
-    dtype: str = "bf16"     # "bf16" or "fp32"
+    dtype: str = "bf16"     # "bf16", "fp32" or "fp8" (FP8 cache, bf16 activations)
     paged: bool = True      # False: identity block table (contiguous cache)
     page_size: int = 64
 
@@ -77,7 +89,8 @@ class Workload:
 
     @property
     def torch_dtype(self) -> torch.dtype:
-        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        """Activations, weights and output."""
+        return torch.float32 if self.dtype == "fp32" else torch.bfloat16
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -99,10 +112,16 @@ WORKLOADS = {
     "tpla_dsv3": Workload("tpla_dsv3", seed=4, batch=32, q_len=1, heads=128,
                           latent_rank=512, rope_dim=64, nope_dim=128, v_dim=128,
                           context=32768, latent_shards=2),
+    "deepseek_v3_fp8": Workload("deepseek_v3_fp8", seed=5, batch=32, q_len=1, heads=128,
+                                latent_rank=512, rope_dim=64, nope_dim=128, v_dim=128,
+                                context=32768, dtype="fp8"),
 }
 
 _TAG_LENS, _TAG_QN, _TAG_QR, _TAG_WUK, _TAG_WUV, _TAG_PERM = 1, 2, 3, 4, 5, 6
 _TAG_SEQ0 = 100
+_TAG_SCALE0 = 200
+FP8_CODE_STD = 32.0                      # std of the values cast to E4M3 codes
+FP8_SCALE_RANGE = (1.0 / 48.0, 1.0 / 24.0)
 
 
 def _gen(seed: int, tag: int) -> torch.Generator:
@@ -157,6 +176,8 @@ def generate(wl: Workload, seq_lens: Optional[Sequence[int]] = None,
         return out
 
     P = wl.page_size
+    if wl.dtype == "fp8":
+        return _fp8_pool(wl, lens, out)
     npages = [pages_of(int(L), P) for L in lens.tolist()]
     total = sum(npages)
     max_pages = max(npages) if npages else 0
@@ -180,6 +201,53 @@ def generate(wl: Workload, seq_lens: Optional[Sequence[int]] = None,
     out["block_table"] = table
     out["num_blocks"] = total
     return out
+
+
+def _fp8_pool(wl: Workload, lens: torch.Tensor, out: dict) -> dict:
+    P, r, dr = wl.page_size, wl.latent_rank, wl.rope_dim
+    B = int(lens.numel())
+    npages = [pages_of(int(L), P) for L in lens.tolist()]
+    total = sum(npages)
+    perm = torch.randperm(total, generator=_gen(wl.seed, _TAG_PERM)).to(torch.int32)
+    table = torch.full((B, max(max(npages) if npages else 0, 1)), -1, dtype=torch.int32)
+    codes = torch.zeros((total, P, r), dtype=torch.uint8)
+    rope = torch.zeros((total, P, dr), dtype=torch.bfloat16)
+    scale = torch.zeros((total, P), dtype=torch.float32)
+    lo, hi = FP8_SCALE_RANGE
+    base = 0
+    for b, L in enumerate(lens.tolist()):
+        n = npages[b]
+        ids = perm[base:base + n]
+        table[b, :n] = ids
+        x = torch.randn((L, wl.row_width), generator=_gen(wl.seed, _TAG_SEQ0 + b),
+                        dtype=torch.float32) * FP8_CODE_STD
+        c = torch.zeros((n * P, r), dtype=torch.uint8)
+        c[:L] = x[:, :r].to(torch.float8_e4m3fn).view(torch.uint8)
+        k = torch.zeros((n * P, dr), dtype=torch.bfloat16)
+        k[:L] = x[:, r:].to(torch.bfloat16)
+        sc = torch.zeros(n * P, dtype=torch.float32)
+        sc[:L] = lo + (hi - lo) * torch.rand(L, generator=_gen(wl.seed, _TAG_SCALE0 + b))
+        codes[ids.long()] = c.view(n, P, r)
+        rope[ids.long()] = k.view(n, P, dr)
+        scale[ids.long()] = sc.view(n, P)
+        base += n
+    out["kv_codes"], out["kv_rope"], out["kv_scale"] = codes, rope, scale
+    out["block_table"] = table
+    out["num_blocks"] = total
+    return out
+
+
+def stored_rows_fp8(inputs: dict, b: int, wl: Workload):
+    """(codes uint8 [L_b, r], stored RoPE key bf16 [L_b, dr], scales [L_b]) of
+    sequence b, gathered from the FP8 pool (layout only, no arithmetic)."""
+    L = int(inputs["seq_lens"][b])
+    P = wl.page_size
+    n = pages_of(L, P)
+    ids = inputs["block_table"][b, :n].long()
+    codes = inputs["kv_codes"][ids].reshape(n * P, wl.latent_rank)[:L]
+    rope = inputs["kv_rope"][ids].reshape(n * P, wl.rope_dim)[:L]
+    scale = inputs["kv_scale"][ids].reshape(n * P)[:L]
+    return codes, rope, scale
 
 
 def logical_cache(inputs: dict, b: int, wl: Workload):

@@ -7,12 +7,13 @@ import numpy as np
 import torch
 
 import mla_latent_kv_21_b200 as M
-from mla_workloads import Workload, generate, logical_cache
-from oracle import mla_oracle
+from mla_workloads import Workload, generate, logical_cache, stored_rows_fp8
+from oracle import fp8_cache, mla_oracle
 
 # bf16 inputs with fp32 accumulation: max-abs <= 2e-2 and rel-Frobenius <= 5e-3;
 # the fp32 workload: rel-Frobenius <= 1e-5.
-TOL = {"bf16": dict(max_abs=2e-2, rel_fro=5e-3), "fp32": dict(max_abs=1e-4, rel_fro=1e-5)}
+TOL = {"bf16": dict(max_abs=2e-2, rel_fro=5e-3), "fp32": dict(max_abs=1e-4, rel_fro=1e-5),
+       "fp8": dict(max_abs=2e-2, rel_fro=5e-3)}  # FP8 cache: against its dequantised values
 
 
 def dims_of(wl: Workload):
@@ -35,8 +36,12 @@ def run_gpu(wl: Workload, inputs: dict, device, kernel=M.MLA_KERNEL_AUTO, num_wo
     out = torch.full((B, wl.q_len, wl.heads, wl.v_dim), float("nan"), dtype=wl.torch_dtype,
                      device=device)
     for _ in range(repeat):
-        plan.run(dev["q_nope"], dev["q_rope"], dev["kv_pool"], dev["block_table"],
-                 dev["seq_lens"], dev["w_uk"], dev["w_uv"], out)
+        if wl.dtype == "fp8":
+            plan.run_fp8(dev["q_nope"], dev["q_rope"], dev["kv_codes"], dev["kv_rope"], dev["kv_scale"],
+                         dev["block_table"], dev["seq_lens"], dev["w_uk"], dev["w_uv"], out)
+        else:
+            plan.run(dev["q_nope"], dev["q_rope"], dev["kv_pool"], dev["block_table"],
+                     dev["seq_lens"], dev["w_uk"], dev["w_uv"], out)
     torch.cuda.synchronize(device)
     status = plan.read_status()
     assert status == expect_status, M.mla_status_string(status)
@@ -51,8 +56,13 @@ def oracle_out(wl: Workload, inputs: dict, batch_indices=None, heads=None) -> np
     bs = list(range(B)) if batch_indices is None else list(batch_indices)
     ckv, kr = {}, {}
     for b in bs:
-        c, k = logical_cache(inputs, b, wl)
-        ckv[b], kr[b] = c.double().numpy(), k.double().numpy()
+        if wl.dtype == "fp8":
+            codes, rope, scale = stored_rows_fp8(inputs, b, wl)
+            ckv[b], kr[b] = fp8_cache.logical_cache_fp8(codes.numpy(), rope.double().numpy(),
+                                                        scale.double().numpy())
+        else:
+            c, k = logical_cache(inputs, b, wl)
+            ckv[b], kr[b] = c.double().numpy(), k.double().numpy()
     return mla_oracle.mla_decode(inputs["q_nope"].double().numpy(),
                                  inputs["q_rope"].double().numpy(), ckv, kr,
                                  inputs["w_uk"].double().numpy(), inputs["w_uv"].double().numpy(),

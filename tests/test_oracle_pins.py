@@ -15,6 +15,7 @@ import math
 import os
 
 import numpy as np
+import torch
 import pytest
 
 from oracle import mla_oracle as mo
@@ -319,3 +320,27 @@ def test_planted_mistakes_are_caught(monkeypatch, target, mutant):
     monkeypatch.setattr(mo, target, mutant)
     got = mo.mla_decode(*prob, scale=scale, latent_shards=2)
     assert np.abs(got - want).max() > 1e-6
+
+
+# ---------------------------------------------------------------------------
+# FP8 cache format: the oracle's E4M3 decoder (written from the bit fields)
+# against torch's own float8_e4m3fn conversion, every code.
+# ---------------------------------------------------------------------------
+def test_e4m3_decoder_matches_torch_on_every_code():
+    from oracle.fp8_cache import e4m3_table
+    ours = e4m3_table()
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan) and nan.sum() == 2  # 0x7F and 0xFF
+    assert np.array_equal(ours[~nan], ref[~nan])
+    assert ours[0x7E] == 448.0 and ours[0x01] == 2.0 ** -9 and ours[0x38] == 1.0
+
+
+def test_fp8_logical_cache_scales_codes_and_rope():
+    from oracle.fp8_cache import logical_cache_fp8
+    codes = np.array([[0x38, 0xC0, 0x00], [0x40, 0x01, 0xB8]], dtype=np.uint8)   # 1, -2, 0 / 2, 2^-9, -1
+    rope = np.array([[1.0, -3.0], [0.5, 2.0]])
+    scales = np.array([0.25, 4.0])
+    ckv, kr = logical_cache_fp8(codes, rope, scales)
+    assert np.array_equal(ckv, [[0.25, -0.5, 0.0], [8.0, 4.0 * 2.0 ** -9, -4.0]])
+    assert np.array_equal(kr, [[0.25, -0.75], [2.0, 8.0]])
