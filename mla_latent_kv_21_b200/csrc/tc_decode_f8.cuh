@@ -5,9 +5,9 @@
 // 64, 64-token pages, up to 128 query rows, one latent shard.
 //
 // The CTA pair, its split of query rows and tokens, the group of 4 pages, the
-// tensor-memory layout, the softmax and the segment epilogue are those of the
-// bf16 kernel (tc_decode.cuh). What changes is what crosses HBM and how it is
-// multiplied:
+// tensor-memory layout, the online softmax and the segment epilogue are those
+// of the bf16 kernel (tc_decode.cuh). What changes is what crosses HBM, how it
+// is multiplied, and the softmax's code shape:
 //
 //   QK  per group five ring items instead of nine: four of 128 tokens x 128
 //       code bytes (one 128-column chunk of cKV) and the RoPE chunk (128 tokens
@@ -23,6 +23,13 @@
 //       P' = p_t * s_t goes to shared memory as P'_hi = e4m3(P') and P'_lo =
 //       e5m2(P' - P'_hi) and each K step of 32 tokens takes two kind::f8f6f4
 //       MMAs (P'_hi . code and P'_lo . code), so O accumulates sum_t p_t cKV_t.
+//   softmax  the per-element work is about three times the bf16 kernel's, so
+//       both passes (row max; P, P' and its split) walk a thread's 128 columns
+//       32 at a time through one copy of their loop body, reading S from
+//       tensor memory twice, and P' goes to shared memory 32 tokens at a time:
+//       unrolled over 128 columns the code outgrows the instruction cache.
+//       Each token half has its own P' buffer (the QK ring has three slots to
+//       make room), so neither half waits for PV of the other's tokens.
 //
 // The two-term splits keep the operands near bf16 precision (the e4m3 term
 // leaves a residual below 2^-4 of the value, which the e5m2 term carries to
@@ -65,10 +72,10 @@ constexpr uint32_t kQChunkBytes = 64 * 128;           // 64 rows x 128 B
 constexpr uint32_t kQBytes = kQChunks * kQChunkBytes;  // 72 KB
 constexpr uint32_t kQRowBytes = 1152;                 // workspace query row: hi 512 | lo 512 | RoPE 128
 constexpr uint32_t kSlotBytes = 16384;                // 128 tokens x 128 B
-constexpr int kQkSlots = 4;
+constexpr int kQkSlots = 3;
 constexpr int kVSlots = 4;
 constexpr uint32_t kPHalfBytes = 64 * 128;            // one token half of P': 64 rows x 128 tokens
-constexpr uint32_t kPRegion = 2 * kPHalfBytes;        // P'_hi and P'_lo of the current token half
+constexpr uint32_t kPRegion = 2 * kPHalfBytes;        // P'_hi and P'_lo of one token half (two buffers)
 constexpr uint32_t kScaleBytes = kGroupPages * 64 * 4;  // token scales of one group
 constexpr int kScaleBufs = 4;                         // groups of scales in flight (producer runs ahead)
 
@@ -77,7 +84,7 @@ struct Smem {
   static constexpr uint32_t qk = q + kQBytes;
   static constexpr uint32_t v = qk + kQkSlots * kSlotBytes;
   static constexpr uint32_t p = v + kVSlots * kSlotBytes;
-  static constexpr uint32_t xch = p + kPRegion;        // float [2][128] row max + [128] l
+  static constexpr uint32_t xch = p + 2 * kPRegion;    // float [2][128] row max + [128] l
   static constexpr uint32_t sc = xch + 3 * 128 * 4;    // float [kScaleBufs][256] token scales
   static constexpr uint32_t bars = sc + kScaleBufs * kScaleBytes;
   static constexpr uint32_t nbars = 48;
@@ -388,7 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         MLA_TRACE_EV(w, 0, tc::EV_PV_START, gi);
         for (int th = 0; th < 2 && ok; ++th) {
           if (th == 1) {
-            ok = mbar_wait(bar(B_P_FULL_HI), gi & 1);  // P' of pages 2, 3 in the shared buffer
+            ok = mbar_wait(bar(B_P_FULL_HI), gi & 1);  // P' of pages 2, 3 in its buffer
             if (!ok) break;
           }
           for (int nb = 0; nb < 2 && ok; ++nb, ++vc) {
@@ -398,11 +405,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             MLA_TRACE_CHUNK(w, 0, 3, vc);
             tc_fence_after();
             const uint64_t vd = v_desc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+            const uint64_t pd = p_desc0 + (uint64_t)((th * kPRegion) >> 4);  // this token half's P
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {  // K = 128 tokens = 4 x 32; V steps 32 rows x 128 B
-              mma_f8(tbase + kTmemO + 128 * nb, p_desc0 + (uint64_t)(2 * ks), vd + (uint64_t)(256 * ks),
+              mma_f8(tbase + kTmemO + 128 * nb, pd + (uint64_t)(2 * ks), vd + (uint64_t)(256 * ks),
                      idesc_hi, (g.first && th == 0 && ks == 0) ? 0u : 1u);
-              mma_f8(tbase + kTmemO + 128 * nb, p_desc0 + (uint64_t)((kPHalfBytes >> 4) + 2 * ks),
+              mma_f8(tbase + kTmemO + 128 * nb, pd + (uint64_t)((kPHalfBytes >> 4) + 2 * ks),
                      vd + (uint64_t)(256 * ks), idesc_lo, 1u);
             }
             commit_both(B_V_FREE + slot);
@@ -459,17 +467,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       wait(B_S_FULL + sb, (gi >> 1) & 1);
       if (lq == 0) MLA_TRACE_EV(w, rank, tc::EV_S_READY, gi);
       if (ok) tc_fence_after();
-      uint32_t r[128];
-      if (ok) {
-#pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32)
-          tmem_ld32(tbase + lane_off + sb * 128 + c0, *reinterpret_cast<uint32_t(*)[32]>(r + c0));
-        tmem_wait_ld();
-      }
-      if (ok) tc_fence_before();
-      __syncwarp();
-      if (ok && lane == 0) arrive_leader(B_S_FREE + sb);
-      // S holds score / s_t: multiply column t by its token scale
+      const uint32_t s_col = tbase + lane_off + sb * 128;  // this thread's 128 S columns
+      // S holds score / s_t: column t is multiplied by its token scale
       wait(B_SC_FULL + gi % kScaleBufs, (gi / kScaleBufs) & 1);
       float* sc_tab = scales + (gi % kScaleBufs) * (kScaleBytes / 4);
       const float* sct = sc_tab + 128 * half;
@@ -485,27 +484,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       if (lq == 0) MLA_TRACE_EV(w, rank, tc::EV_PASS1, gi);
-      if (ok) {
+      // 32 S columns from tensor memory times their token scales; keys masked
+      // for this row (past the group or the causal limit) become -inf
+      auto load_scaled = [&](int c0, uint32_t (&r)[32]) {
+        tmem_ld32(s_col + c0, r);
+        tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 128; j += 4) {
-          const float4 s4 = *reinterpret_cast<const float4*>(sct + j);
+        for (int j = 0; j < 32; j += 4) {
+          const float4 s4 = *reinterpret_cast<const float4*>(sct + c0 + j);
           r[j] = __float_as_uint(__uint_as_float(r[j]) * s4.x);
           r[j + 1] = __float_as_uint(__uint_as_float(r[j + 1]) * s4.y);
           r[j + 2] = __float_as_uint(__uint_as_float(r[j + 2]) * s4.z);
           r[j + 3] = __float_as_uint(__uint_as_float(r[j + 3]) * s4.w);
         }
-      }
-      if (nvis < 128) {
+        if (nvis < c0 + 32) {
 #pragma unroll
-        for (int j = 0; j < 128; ++j)
-          if (j >= nvis) r[j] = 0xff800000u;
-      }
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j >= nvis) r[j] = 0xff800000u;
+        }
+      };
+      // Both passes walk the 128 columns 32 at a time through one copy of
+      // their loop body and read tensor memory twice: a fully unrolled
+      // 128-column pass is more code than the instruction cache holds.
       float mx0 = -INFINITY, mx1 = -INFINITY;
       if (ok) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t r[32];
+          load_scaled(c0, r);
 #pragma unroll
-        for (int j = 0; j < 128; j += 2) {
-          mx0 = fmaxf(mx0, __uint_as_float(r[j]));
-          mx1 = fmaxf(mx1, __uint_as_float(r[j + 1]));
+          for (int j = 0; j < 32; j += 2) {
+            mx0 = fmaxf(mx0, __uint_as_float(r[j]));
+            mx1 = fmaxf(mx1, __uint_as_float(r[j + 1]));
+          }
         }
       }
       const float mt_own = fmaxf(mx0, mx1) * p.scale_log2;
@@ -521,29 +532,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool rescale = mu != m && m != -INFINITY;
       if (rescale) alpha = ex2_approx(m - mu);
       m = mu;
-      // P = 2^(score * scale - m); P' = P * s_t split into e4m3 + e5m2 bytes;
-      // the row sum takes P itself
-      uint32_t ph[32], pl[32];
-      float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
-      const float nmu = mu == -INFINITY ? 0.f : -mu;
-#pragma unroll
-      for (int j = 0; j < 128; j += 4) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, nmu));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, nmu));
-        const float p2 = ex2_approx(fmaf(__uint_as_float(r[j + 2]), p.scale_log2, nmu));
-        const float p3 = ex2_approx(fmaf(__uint_as_float(r[j + 3]), p.scale_log2, nmu));
-        ps0 += p0; ps1 += p1; ps2 += p2; ps3 += p3;
-        // a key masked for this row has P = 0 (score -inf) and a finite table entry
-        const float4 s4 = *reinterpret_cast<const float4*>(sct + j);
-        split4(p0 * s4.x, p1 * s4.y, p2 * s4.z, p3 * s4.w, ph[j >> 2], pl[j >> 2]);
-      }
-      // the zeroing stores above (generic proxy) come before the next bulk copy
-      // into this table (async proxy)
-      if (ok) fence_proxy_async_smem();
-      __syncwarp();
-      if (ok && lane == 0) mbar_arrive_local(bar(B_SC_FREE + gi % kScaleBufs));
-      l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
-      if (lq == 0) MLA_TRACE_EV(w, rank, tc::EV_PASS2, gi);
       auto rescale_o = [&]() {
         tc_fence_after();
 #pragma unroll 1
@@ -557,37 +545,63 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
       };
-      // P'_hi / P'_lo rows -> shared memory, K-major 128-byte swizzle: row
-      // rloc, this thread's 128 tokens as one 128-byte row of each
-      auto write_p = [&](uint8_t* region) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          *reinterpret_cast<uint4*>(region + sw128(rloc, u)) =
-              make_uint4(ph[4 * u], ph[4 * u + 1], ph[4 * u + 2], ph[4 * u + 3]);
-          *reinterpret_cast<uint4*>(region + kPHalfBytes + sw128(rloc, u)) =
-              make_uint4(pl[4 * u], pl[4 * u + 1], pl[4 * u + 2], pl[4 * u + 3]);
-        }
-      };
       // O is rescaled (after the previous group's PV) before this group's PV
-      // adds to it; one P' buffer holds pages 0, 1 and then pages 2, 3
+      // adds to it: B_P_FULL counts half 0's P' writes and half 1's rescale.
+      // Each token half has its own P' buffer, free once the previous group's
+      // PV of that half is done.
       if (!g.first && __any_sync(0xffffffffu, rescale)) wait(B_PV_DONE, (gi - 1) & 1);
       if (ok && !g.first && __any_sync(0xffffffffu, rescale)) rescale_o();
-      if (half == 0) {
-        if (gi >= 1) wait(B_P_FREE_HI, (gi - 1) & 1);
-      } else {
+      if (half == 1) {
         if (ok) tc_fence_before();
         __syncwarp();
         if (ok && lane == 0) arrive_leader(B_P_FULL);
-        wait(B_P_FREE_LO, gi & 1);
       }
+      if (gi >= 1) wait(half == 0 ? B_P_FREE_LO : B_P_FREE_HI, (gi - 1) & 1);
       if (lq == 0) MLA_TRACE_EV(w, rank, tc::EV_PBUF_FREE, gi);
+      // P = 2^(score * scale - m); P' = P * s_t split into e4m3 + e5m2 bytes,
+      // written 32 tokens at a time into row rloc of this half's P' buffer
+      // (K-major, 128-byte swizzle: 16-byte units c0 / 16 and c0 / 16 + 1);
+      // the row sum takes P itself
+      uint8_t* pbuf = gbase + L::p + half * kPRegion;
+      float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
+      const float nmu = mu == -INFINITY ? 0.f : -mu;
       if (ok) {
-        write_p(gbase + L::p);
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t r[32];
+          load_scaled(c0, r);
+          uint32_t ph[8], pl[8];
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, nmu));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, nmu));
+            const float p2 = ex2_approx(fmaf(__uint_as_float(r[j + 2]), p.scale_log2, nmu));
+            const float p3 = ex2_approx(fmaf(__uint_as_float(r[j + 3]), p.scale_log2, nmu));
+            ps0 += p0; ps1 += p1; ps2 += p2; ps3 += p3;
+            // a key masked for this row has P = 0 (score -inf) and a finite table entry
+            const float4 s4 = *reinterpret_cast<const float4*>(sct + c0 + j);
+            split4(p0 * s4.x, p1 * s4.y, p2 * s4.z, p3 * s4.w, ph[j >> 2], pl[j >> 2]);
+          }
+          const int u0 = c0 >> 4;
+          *reinterpret_cast<uint4*>(pbuf + sw128(rloc, u0)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+          *reinterpret_cast<uint4*>(pbuf + sw128(rloc, u0 + 1)) = make_uint4(ph[4], ph[5], ph[6], ph[7]);
+          *reinterpret_cast<uint4*>(pbuf + kPHalfBytes + sw128(rloc, u0)) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+          *reinterpret_cast<uint4*>(pbuf + kPHalfBytes + sw128(rloc, u0 + 1)) =
+              make_uint4(pl[4], pl[5], pl[6], pl[7]);
+        }
+        // P' (and the table's zeroing stores) before the MMAs and the next bulk
+        // copy into the table (async proxy); the S reads before QK reuses S
         fence_proxy_async_smem();
         tc_fence_before();
       }
+      l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
+      if (lq == 0) MLA_TRACE_EV(w, rank, tc::EV_PASS2, gi);
       __syncwarp();
-      if (ok && lane == 0) arrive_leader(half == 0 ? B_P_FULL : B_P_FULL_HI);
+      if (ok && lane == 0) {
+        arrive_leader(B_S_FREE + sb);
+        mbar_arrive_local(bar(B_SC_FREE + gi % kScaleBufs));
+        arrive_leader(half == 0 ? B_P_FULL : B_P_FULL_HI);
+      }
       if (lq == 0) MLA_TRACE_EV(w, rank, tc::EV_P_DONE, gi);
 
       if (g.last_of_segment()) {
