@@ -22,7 +22,10 @@
  *   kv_cache [num_blocks, page_size, r + d_rope]; columns [0, r) are cKV,
  *            columns [r, r + d_rope) the decoupled RoPE key (after RoPE)
  *   block_table int32 [B, block_table_stride]; entry (b, i) is the block that
- *            holds tokens [i*page_size, (i+1)*page_size) of sequence b
+ *            holds tokens [i*page_size, (i+1)*page_size) of sequence b. The
+ *            slots of a sequence's last block past L_b are read (whole pages
+ *            move) and their cKV weighted by exactly 0: their cKV columns must
+ *            hold finite values (any; 0 * NaN would still be NaN).
  *   seq_lens int32 [B], L_b counts the Lq query tokens (they are the newest
  *            Lq cache rows; query t sees keys j <= L_b - Lq + t)
  *   w_uk     [H, d_nope, r]     w_uv [H, r, d_v]
@@ -171,8 +174,10 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan,
  *   kv_rope  bf16  [num_blocks, page_size, d_rope] RoPE key divided by s_t
  *   kv_scale fp32  [num_blocks, page_size]      s_t, so that cKV_t = s_t * code_t
  *                                               and k_rope_t = s_t * kv_rope_t
- * (kv_scale 16-byte aligned). Every other argument, the workspace and the
- * errors are as for mla_decode_run_ex. The tensor-core MMAs take e4m3 / e5m2
+ * (kv_scale 16-byte aligned). As for the bf16 cache, the codes of slots past
+ * L_b must be finite (no 0x7F or 0xFF); their RoPE keys and scales may hold
+ * anything. Every other argument, the workspace and the errors are as for
+ * mla_decode_run_ex. The tensor-core MMAs take e4m3 / e5m2
  * operands: the absorbed query and P * s_t each as an e4m3 value plus an e5m2
  * correction, so that the result stays within the bf16 tolerance of the
  * dequantised cache; P * s_t must stay below 448 (s_t <= 1.75). */
