@@ -121,8 +121,10 @@ typedef struct mla_plan* mla_plan_t; /* opaque, library-owned host object */
  * the device lengths passed to run may differ as long as each stays in
  * [Lq, block_table_stride * page_size]: the split partition is recomputed
  * on the device every run, so only balance (not correctness) depends on the
- * plan-time lengths. On success *plan_out receives a new plan (free it with
- * mla_plan_destroy) and *workspace_bytes the workspace size run needs. */
+ * plan-time lengths. batch >= 1: an empty batch has nothing to decode and is
+ * refused with MLA_ERR_INVALID_ARG. On success *plan_out receives a new plan
+ * (free it with mla_plan_destroy) and *workspace_bytes the workspace size run
+ * needs. */
 mla_status_t mla_decode_plan(const mla_dims_t* dims, int32_t batch,
                              const int32_t* seq_lens_host, int32_t num_sms,
                              mla_plan_t* plan_out, size_t* workspace_bytes);

@@ -172,6 +172,10 @@ def test_workspace_holds_partials_for_every_slot():
      L.MLA_KERNEL_TCGEN05_LSPLIT, L.MLA_ERR_UNSUPPORTED),
     # unknown kernel kind
     (dict(), 7, L.MLA_ERR_INVALID_ARG),
+    # the FP8 cache runs on the tcgen05 decode kernel only, with one latent shard
+    (dict(dtype="fp8"), L.MLA_KERNEL_SIMT, L.MLA_ERR_UNSUPPORTED),
+    (dict(dtype="fp8"), L.MLA_KERNEL_TCGEN05_LSPLIT, L.MLA_ERR_UNSUPPORTED),
+    (dict(dtype="fp8", latent_shards=2), L.MLA_KERNEL_AUTO, L.MLA_ERR_UNSUPPORTED),
 ])
 def test_plan_rejects_unsupported_kernel_choices(kw, kernel, status):
     with pytest.raises(L.MlaError) as e:
@@ -189,5 +193,24 @@ def test_plan_reports_kernel_and_launches(kernel):
         assert info.kernel == want
         assert info.launches_per_run == 3
         assert info.workspace_bytes == ws > 0
+    finally:
+        L.mla_plan_destroy(plan)
+
+
+def test_plan_rejects_an_empty_batch():
+    with pytest.raises(L.MlaError) as e:
+        L.mla_decode_plan(_dims(), [], num_sms=148)
+    assert e.value.status == L.MLA_ERR_INVALID_ARG
+
+
+def test_fp8_plan_uses_tcgen05_and_bf16_run_refuses_it():
+    plan, ws = L.mla_decode_plan_ex(_dims(dtype="fp8"), [4000, 65], num_sms=148, kernel=L.MLA_KERNEL_AUTO)
+    try:
+        info = L.mla_plan_get_info(plan)
+        assert info.kernel == L.MLA_KERNEL_TCGEN05 and info.launches_per_run == 3
+        fake = 1 << 20  # never dereferenced: the dtype check comes before any launch
+        with pytest.raises(L.MlaError) as e:
+            L.mla_decode_run(plan, fake, fake, fake, 1, fake, 1, fake, fake, fake, fake, fake, ws, 0)
+        assert e.value.status == L.MLA_ERR_INVALID_ARG
     finally:
         L.mla_plan_destroy(plan)
