@@ -70,3 +70,24 @@ def test_two_plans_on_two_streams(cuda_device):
         assert plan.read_status() == 0
         assert torch.equal(out.cpu().view(torch.int16), solo.view(torch.int16)), wl.name
         plan.close()
+
+
+def test_tail_slots_may_hold_any_rope_and_finite_ckv(cuda_device):
+    # slots past a sequence's length in its last page are read (whole pages
+    # move) but weighted by exactly 0: NaN RoPE keys (masked scores) and large
+    # finite cKV there leave the output bit-identical
+    wl = WORKLOADS["deepseek_v3"]
+    inputs = generate(wl, seq_lens=[1, 63, 65, 200])
+    pool = inputs["kv_pool"].clone()
+    P, r = wl.page_size, wl.latent_rank
+    for b, L in enumerate(inputs["seq_lens"].tolist()):
+        npg = -(-L // P)
+        blk = int(inputs["block_table"][b, npg - 1])
+        t0 = L - (npg - 1) * P
+        pool[blk, t0:, :r] = 3.0e4
+        pool[blk, t0:, r:] = float("nan")
+    clean, _ = run_gpu(wl, inputs, cuda_device)
+    dirty, _ = run_gpu(wl, dict(inputs, kv_pool=pool), cuda_device)
+    assert torch.isfinite(dirty.float()).all()
+    assert torch.equal(clean, dirty)
+

@@ -6,8 +6,11 @@ measures the GPU path's own error (the query and P split into e4m3 + e5m2
 operands, the fp16 partials, bf16 output) against the bf16 tolerance.
 """
 
+import dataclasses
+
 import numpy as np
 import pytest
+import torch
 
 from mla_workloads import WORKLOADS, generate
 
@@ -16,6 +19,8 @@ from harness import assert_close, oracle_out, run_gpu
 pytestmark = pytest.mark.gpu
 
 WL = WORKLOADS["deepseek_v3_fp8"]
+# the Kimi-K2 MTP shape (64 heads, two query tokens with the causal rule) over the FP8 cache
+MTP = dataclasses.replace(WORKLOADS["kimi_k2_mtp"], name="kimi_k2_mtp_fp8", dtype="fp8")
 
 
 @pytest.mark.parametrize("lens", [[1, 63, 64, 65, 130, 200, 700], [2048], [3000, 1, 257]])
@@ -40,3 +45,38 @@ def test_full_size_sampled_parity(cuda_device):
     for b, h in [(0, 0), (13, 77), (31, 127)]:
         ref = oracle_out(WL, inputs, [b], [h])[0, :, 0]
         assert_close(got[b, :, h], ref, WL.dtype, f"b={b} h={h}")
+
+
+@pytest.mark.parametrize("lens", [[2, 65, 300, 1030], [129, 3]])
+def test_mtp_parity(cuda_device, lens):
+    # row t of a sequence sees keys j <= L - 2 + t: a segment holding only the
+    # last key has a row that sees nothing there
+    inputs = generate(MTP, seq_lens=lens)
+    got, _ = run_gpu(MTP, inputs, cuda_device, num_workers=5)
+    assert_close(got.double().numpy(), oracle_out(MTP, inputs), MTP.dtype, f"mtp fp8 {lens}")
+
+
+def _poison_tail_slots(inputs, wl):
+    """Slots past each sequence's length in its last page: codes set to the
+    largest finite e4m3 value (0x7E = 448), RoPE keys and scales to NaN."""
+    P = wl.page_size
+    codes, rope, scale = inputs["kv_codes"].clone(), inputs["kv_rope"].clone(), inputs["kv_scale"].clone()
+    for b, L in enumerate(inputs["seq_lens"].tolist()):
+        npg = -(-L // P)
+        blk = int(inputs["block_table"][b, npg - 1])
+        t0 = L - (npg - 1) * P
+        codes[blk, t0:] = 0x7E
+        rope[blk, t0:] = float("nan")
+        scale[blk, t0:] = float("nan")
+    return dict(inputs, kv_codes=codes, kv_rope=rope, kv_scale=scale)
+
+
+def test_tail_slots_may_hold_any_scale_and_rope(cuda_device):
+    # a key past the sequence is weighted by exactly 0, its scale is replaced
+    # by 0 in the kernel, its score is masked: the output cannot change
+    inputs = generate(WL, seq_lens=[1, 63, 65, 200])
+    clean, _ = run_gpu(WL, inputs, cuda_device)
+    dirty, _ = run_gpu(WL, _poison_tail_slots(inputs, WL), cuda_device)
+    assert torch.isfinite(dirty.float()).all()
+    assert torch.equal(clean, dirty)
+
