@@ -90,23 +90,30 @@ def step_work(wl, lens):
                 exps=rows * sum_l * S)
 
 
-def kernel_source_digest():
+# The sources a recorded traffic figure depends on: the decode kernel's own
+# headers and the file that configures its launch (files of other kernels do
+# not change what this one reads and writes).
+_DECODE_SOURCES = ["common.cuh", "sm100_ptx.cuh", "tc_decode.cuh", "mla_decode_api.cu"]
+TRAFFIC_SOURCES = {"bf16": _DECODE_SOURCES, "fp8": _DECODE_SOURCES + ["tc_decode_f8.cuh"]}
+
+
+def kernel_source_digest(dtype="bf16"):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_latent_kv_21_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in sorted(TRAFFIC_SOURCES.get(dtype, os.listdir(csrc))):
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload, kernel):
+def recorded_traffic(workload, kernel, dtype="bf16"):
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
     ent = rec.get(workload, {}).get(kernel)
-    if not ent or ent.get("source_digest") != kernel_source_digest():
+    if not ent or ent.get("source_digest") != kernel_source_digest(dtype):
         return None
     return ent.get("bytes_per_launch")
 
@@ -558,7 +565,7 @@ def main():
                 "achieved": work["decode_flops"] / dec_s / 1e12, "peak": flop_peak,
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = recorded_traffic(wl.name, kname)
+    roof["traffic"] = recorded_traffic(wl.name, kname, wl.dtype)
     roof["kernel"] = f"decode_{kname}"
     roof["peak_source"] = f"{peaks_kind} ({flop_kind} for FLOPs)"
     roof["decode_us"] = dec_s * 1e6

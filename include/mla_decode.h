@@ -179,10 +179,12 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan,
  * (kv_scale 16-byte aligned). As for the bf16 cache, the codes of slots past
  * L_b must be finite (no 0x7F or 0xFF); their RoPE keys and scales may hold
  * anything. Every other argument, the workspace and the errors are as for
- * mla_decode_run_ex. The tensor-core MMAs take e4m3 / e5m2
- * operands: the absorbed query and P * s_t each as an e4m3 value plus an e5m2
- * correction, so that the result stays within the bf16 tolerance of the
- * dequantised cache; P * s_t must stay below 448 (s_t <= 1.75). */
+ * mla_decode_run_ex. The tensor-core MMAs take e4m3 / e5m2 operands: the
+ * absorbed query as an e4m3 value plus an e5m2 correction, and P * s_t, scaled
+ * per group of 256 keys by a power of two into e4m3's normal range, as two
+ * e4m3 terms; the result stays within twice the bf16 tolerance of the
+ * dequantised cache. s_t must be positive and finite for every visible key
+ * (any magnitude). */
 mla_status_t mla_decode_run_fp8(mla_plan_t plan,
                                 const void* q_nope, const void* q_rope,
                                 const void* kv_codes, const void* kv_rope, const float* kv_scale,

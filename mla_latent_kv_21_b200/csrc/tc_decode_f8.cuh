@@ -20,9 +20,13 @@
 //       table of scales (one 1 KB bulk copy per group).
 //   PV  the cached codes themselves are V: V items of 128 tokens x 128 code
 //       bytes (one column block per CTA), four per group instead of eight.
-//       P' = p_t * s_t goes to shared memory as P'_hi = e4m3(P') and P'_lo =
-//       e5m2(P' - P'_hi) and each K step of 32 tokens takes two kind::f8f6f4
-//       MMAs (P'_hi . code and P'_lo . code), so O accumulates sum_t p_t cKV_t.
+//       P' = 2^kp * p_t * s_t goes to shared memory as P'_hi = e4m3(P') and
+//       P'_lo = e4m3(P' - P'_hi) and each K step of 32 tokens takes two
+//       kind::f8f6f4 MMAs (P'_hi . code and P'_lo . code), so O accumulates
+//       2^kp sum_t p_t cKV_t. The power of two 2^kp, chosen per group from the
+//       group's largest scale, puts the largest weights near 1 (in e4m3's
+//       normal range) and is carried by O and the row sum like a shift of
+//       the running max.
 //   softmax  the per-element work is about three times the bf16 kernel's, so
 //       both passes (row max; P, P' and its split) walk a thread's 128 columns
 //       32 at a time through one copy of their loop body, reading S from
@@ -31,10 +35,11 @@
 //       Each token half has its own P' buffer (the QK ring has three slots to
 //       make room), so neither half waits for PV of the other's tokens.
 //
-// The two-term splits keep the operands near bf16 precision (the e4m3 term
-// leaves a residual below 2^-4 of the value, which the e5m2 term carries to
-// within 2^-3 of itself) while the cache bytes per token fall from 1152 to
-// 644.
+// The two-term splits keep the operands near bf16 precision while the cache
+// bytes per token fall from 1152 to 644: the e4m3 term leaves a residual below
+// 2^-4 of the value, which the query's e5m2 term (any magnitude) carries to
+// within 2^-3 of itself and P's e4m3 term (P' near 1) to within 2^-4, or to an
+// absolute 2^-10 when the residual is below e4m3's normal range.
 //
 // Sources: as tc_decode.cuh (TPLA abstract, TransMLA abstract, pith.science
 // verdict record for 2502.07864); the FP8 cache itself is a format of this
@@ -84,8 +89,8 @@ struct Smem {
   static constexpr uint32_t qk = q + kQBytes;
   static constexpr uint32_t v = qk + kQkSlots * kSlotBytes;
   static constexpr uint32_t p = v + kVSlots * kSlotBytes;
-  static constexpr uint32_t xch = p + 2 * kPRegion;    // float [2][128] row max + [128] l
-  static constexpr uint32_t sc = xch + 3 * 128 * 4;    // float [kScaleBufs][256] token scales
+  static constexpr uint32_t xch = p + 2 * kPRegion;    // float [2][128] row max, [128] l, [2][4] scale max
+  static constexpr uint32_t sc = xch + 3 * 128 * 4 + 2 * 4 * 4;  // float [kScaleBufs][256] token scales
   static constexpr uint32_t bars = sc + kScaleBufs * kScaleBytes;
   static constexpr uint32_t nbars = 48;
   static constexpr uint32_t misc = bars + nbars * 8;   // tmem slot, abort flag
@@ -129,13 +134,15 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t
 }
 
 // (P_hi, P_lo) bytes of four values: two words, byte j = value j. The values
-// go to f16 first (11 significant bits, far below the e5m2 residual's step);
-// hi = e4m3(x), lo = e5m2(x - hi), the difference taken exactly in f16.
+// go to f16 first (11 significant bits, below the residual's step); hi =
+// e4m3(x), lo = e4m3(x - hi), the difference taken exactly in f16. The P pass
+// scales P' into e4m3's normal range, where a residual of at least 2^-6 keeps
+// four significant bits and a smaller one an absolute step of 2^-9.
 __device__ __forceinline__ void split4(float a, float b, float c, float d, uint32_t& hi, uint32_t& lo) {
   const uint32_t x01 = ptx::cvt_f16x2(a, b), x23 = ptx::cvt_f16x2(c, d);
   const uint32_t h01 = ptx::e4m3x2_of_f16x2(x01), h23 = ptx::e4m3x2_of_f16x2(x23);
-  const uint32_t l01 = ptx::e5m2x2_of_f16x2(ptx::sub_f16x2(x01, ptx::f16x2_of_e4m3x2(h01)));
-  const uint32_t l23 = ptx::e5m2x2_of_f16x2(ptx::sub_f16x2(x23, ptx::f16x2_of_e4m3x2(h23)));
+  const uint32_t l01 = ptx::e4m3x2_of_f16x2(ptx::sub_f16x2(x01, ptx::f16x2_of_e4m3x2(h01)));
+  const uint32_t l23 = ptx::e4m3x2_of_f16x2(ptx::sub_f16x2(x23, ptx::f16x2_of_e4m3x2(h23)));
   hi = h01 | (h23 << 16);
   lo = l01 | (l23 << 16);
 }
@@ -381,7 +388,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------ PV MMA issuer --
     if (rank == 0 && lane == 0) {
       const uint32_t idesc_hi = kIdescBase | kMnMajorB;
-      const uint32_t idesc_lo = kIdescBase | kMnMajorB | kE5M2A;
+      const uint32_t idesc_lo = kIdescBase | kMnMajorB;  // P'_lo is e4m3 too
       const uint64_t p_desc0 = smem_desc_sw128(base + L::p, 16, 1024);
       const uint64_t v_desc0 = smem_desc_sw128(base + L::v, kSlotBytes, 1024);
       bool ok = true;
@@ -451,6 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool have = g.init(p, w);
     int gi = 0;
     float m = -INFINITY, l = 0.f;
+    int kp = 0;                                    // P' is held as 2^kp * P * s_t
     while (have) {
       if (g.first) { m = -INFINITY; l = 0.f; }
       const int sb = gi & 1;
@@ -472,16 +480,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       wait(B_SC_FULL + gi % kScaleBufs, (gi / kScaleBufs) & 1);
       float* sc_tab = scales + (gi % kScaleBufs) * (kScaleBytes / 4);
       const float* sct = sc_tab + 128 * half;
+      float* xsmax = xch + 3 * 128 + (gi & 1) * 4;  // [4] per-warp largest scale of this group
       if (ok) {
         // entries of keys past the sequence (or of pages the group lacks) hold
         // whatever the pool or an older group left there: zero them, so that a
         // masked key's P' = 0 * s is 0 whatever it held; the named barrier
-        // below orders these stores before the P pass reads the table
+        // below orders these stores before the P pass reads the table. The
+        // largest valid scale of the group goes to xsmax (scales are > 0, so
+        // their bits order as unsigned integers).
+        uint32_t smax_bits = 0u;
 #pragma unroll
         for (int e = lq; e < 4 * 64; e += 128) {
           const int q = e >> 6;
           if (q >= g.npages || (int64_t)(g.page + q) * 64 + (e & 63) >= Lb) sc_tab[e] = 0.f;
+          else smax_bits = max(smax_bits, __float_as_uint(sc_tab[e]));
         }
+        smax_bits = __reduce_max_sync(0xffffffffu, smax_bits);
+        if (lane == 0) xsmax[warp & 3] = __uint_as_float(smax_bits);
       }
       if (lq == 0) MLA_TRACE_EV(w, rank, tc::EV_PASS1, gi);
       // 32 S columns from tensor memory times their token scales; keys masked
@@ -528,10 +543,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float mt = fmaxf(mt_own, xmax[lq ^ 64]);
       float mu = m;
       if (m == -INFINITY || mt > m + kRescaleThreshold) mu = fmaxf(mt, m);
+      // P' is kept as 2^kp * P * s_t with 2^kp * s_max <= 1.75, so that with
+      // P <= 2^8 (the lazy max) it stays below e4m3's 448 and the group's
+      // largest weights sit near 1, in e4m3's normal range; kp only falls
+      // within a segment. O and l carry the same 2^kp: the exponent offset is
+      // m - kp, and a change of either rescales them like a new max.
+      const float smax = fmaxf(fmaxf(xsmax[0], xsmax[1]), fmaxf(xsmax[2], xsmax[3]));
+      int kg = smax > 0.f ? (int)((__float_as_uint(1.75f / smax) >> 23) & 0xFF) - 127 : kp;
+      kg = kg < -64 ? -64 : (kg > 64 ? 64 : kg);
+      const int kn = g.first ? kg : min(kp, kg);
+      const float off_old = m - (float)kp, off_new = mu - (float)kn;
       float alpha = 1.f;
-      const bool rescale = mu != m && m != -INFINITY;
-      if (rescale) alpha = ex2_approx(m - mu);
+      const bool rescale = m != -INFINITY && off_new != off_old;
+      if (rescale) alpha = ex2_approx(off_old - off_new);
       m = mu;
+      kp = kn;
       auto rescale_o = [&]() {
         tc_fence_after();
 #pragma unroll 1
@@ -558,13 +584,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (gi >= 1) wait(half == 0 ? B_P_FREE_LO : B_P_FREE_HI, (gi - 1) & 1);
       if (lq == 0) MLA_TRACE_EV(w, rank, tc::EV_PBUF_FREE, gi);
-      // P = 2^(score * scale - m); P' = P * s_t split into e4m3 + e5m2 bytes,
+      // P = 2^(score * scale - m + kp); P' = P * s_t split into two e4m3 bytes,
       // written 32 tokens at a time into row rloc of this half's P' buffer
       // (K-major, 128-byte swizzle: 16-byte units c0 / 16 and c0 / 16 + 1);
       // the row sum takes P itself
       uint8_t* pbuf = gbase + L::p + half * kPRegion;
       float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
-      const float nmu = mu == -INFINITY ? 0.f : -mu;
+      const float nmu = mu == -INFINITY ? 0.f : -off_new;
       if (ok) {
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -613,7 +639,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int64_t slot = w + g.b;
         const float lt = l + xl[lq ^ 64];
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        if (ok && half == 0 && row_real) p.lse_part[slot * p.rows + row] = lt > 0.f ? m + log2f(lt) : kEmptyLse;
+        if (ok && half == 0 && row_real) p.lse_part[slot * p.rows + row] = lt > 0.f ? m - (float)kp + log2f(lt) : kEmptyLse;
         if (ok) {
           // a warp's 32 rows x 64 columns per round, transposed through 4 KB
           // of the (idle) P' buffer into whole 128-byte row segments
