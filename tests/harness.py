@@ -12,10 +12,11 @@ from oracle import fp8_cache, mla_oracle
 
 # bf16 inputs with fp32 accumulation: max-abs <= 2e-2 and rel-Frobenius <= 5e-3;
 # the fp32 workload: rel-Frobenius <= 1e-5.
-# FP8 cache, against its dequantised values: the tensor-core operands (the
-# absorbed query, P * s_t) are e4m3 + e5m2 pairs carrying 7 significant bits
-# against bf16's 8, so each relative rounding bound doubles, and so do the
-# bf16 tolerances
+# FP8 cache, against its dequantised values: the absorbed query reaches the
+# tensor cores as an e4m3 + e5m2 pair carrying 7 significant bits against
+# bf16's 8 (P * s_t, an e4m3 pair scaled per group, keeps 8 for its largest
+# weights), so the relative rounding bound of the scores doubles, and so do
+# the bf16 tolerances
 TOL = {"bf16": dict(max_abs=2e-2, rel_fro=5e-3), "fp32": dict(max_abs=1e-4, rel_fro=1e-5),
        "fp8": dict(max_abs=4e-2, rel_fro=1e-2)}
 

@@ -2,8 +2,8 @@
 
 The oracle decodes the cache's E4M3 codes from the format definition and runs
 the non-absorbed fp64 attention on the dequantised values, so the comparison
-measures the GPU path's own error (the query and P split into e4m3 + e5m2
-operands, the fp16 partials, bf16 output) against the bf16 tolerance.
+measures the GPU path's own error (the query as e4m3 + e5m2 and P * s_t as two
+e4m3 terms, the fp16 partials, bf16 output) against the FP8 tolerance.
 """
 
 import dataclasses
