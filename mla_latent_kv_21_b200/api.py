@@ -22,6 +22,7 @@ class DecodePlan:
     def __init__(self, dims: L.mla_dims_t, seq_lens_host: Sequence[int], num_sms: int = 0,
                  kernel: int = L.MLA_KERNEL_AUTO, num_workers: int = 0):
         self.dims = dims
+        self.batch = len(seq_lens_host)
         self.handle, self.workspace_bytes = L.mla_decode_plan_ex(
             dims, list(seq_lens_host), num_sms, kernel, num_workers)
         self.info = L.mla_plan_get_info(self.handle)
@@ -37,17 +38,44 @@ class DecodePlan:
     def segments(self):
         return L.mla_plan_segments(self.handle)
 
+    def _check(self, name, t, dtype, shape) -> None:
+        """One argument's dtype and shape against the plan (None: any extent).
+        The C ABI sees bare pointers, so this is where a mismatch is caught."""
+        if t.dtype != dtype:
+            raise ValueError(f"{name}: dtype {t.dtype}, the plan needs {dtype}")
+        if t.dim() != len(shape) or any(e is not None and e != n for e, n in zip(shape, t.shape)):
+            want = tuple("*" if e is None else e for e in shape)
+            raise ValueError(f"{name}: shape {tuple(t.shape)}, the plan needs {want}")
+
+    def _check_common(self, act, q_nope, q_rope, block_table, seq_lens, w_uk, w_uv, out) -> None:
+        import torch
+        d, B = self.dims, self.batch
+        H, Lq, r, dr, dn, dv = d.num_heads, d.q_len, d.latent_rank, d.rope_dim, d.nope_dim, d.v_dim
+        self._check("q_nope", q_nope, act, (B, Lq, H, dn))
+        self._check("q_rope", q_rope, act, (B, Lq, H, dr))
+        self._check("block_table", block_table, torch.int32, (B, None))
+        self._check("seq_lens", seq_lens, torch.int32, (B,))
+        self._check("w_uk", w_uk, act, (H, dn, r))
+        self._check("w_uv", w_uv, act, (H, r, dv))
+        self._check("out", out, act, (B, Lq, H, dv))
+
     def run(self, q_nope, q_rope, kv_pool, block_table, seq_lens, w_uk, w_uv, out,
             stream: Optional[int] = None, decode_events=None) -> None:
         """All arguments are device tensors laid out as in include/mla_decode.h."""
         import torch
-        if self.workspace is None:
-            self.allocate_workspace(q_nope.device)
+        d = self.dims
+        if d.dtype == L.MLA_FP8_CACHE:
+            raise ValueError("a plan over the FP8 cache runs with run_fp8")
+        act = torch.float32 if d.dtype == L.MLA_FP32 else torch.bfloat16
+        self._check_common(act, q_nope, q_rope, block_table, seq_lens, w_uk, w_uv, out)
+        self._check("kv_pool", kv_pool, act, (None, d.page_size, d.latent_rank + d.rope_dim))
         for name, t in (("q_nope", q_nope), ("q_rope", q_rope), ("kv_pool", kv_pool),
                         ("block_table", block_table), ("seq_lens", seq_lens), ("w_uk", w_uk),
                         ("w_uv", w_uv), ("out", out)):
             if not t.is_cuda or not t.is_contiguous():
                 raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if self.workspace is None:
+            self.allocate_workspace(q_nope.device)
         if stream is None:
             stream = torch.cuda.current_stream(q_nope.device).cuda_stream
         # decode_events: optional (start, stop) raw cudaEvent_t handles (ints)
@@ -62,13 +90,21 @@ class DecodePlan:
                 w_uv, out, stream: Optional[int] = None, decode_events=None) -> None:
         """As run, over an FP8 latent cache (include/mla_decode.h, mla_decode_run_fp8)."""
         import torch
-        if self.workspace is None:
-            self.allocate_workspace(q_nope.device)
+        d = self.dims
+        if d.dtype != L.MLA_FP8_CACHE:
+            raise ValueError("run_fp8 needs a plan made with dtype 'fp8'")
+        self._check_common(torch.bfloat16, q_nope, q_rope, block_table, seq_lens, w_uk, w_uv, out)
+        nb = kv_codes.shape[0] if kv_codes.dim() == 3 else None
+        self._check("kv_codes", kv_codes, torch.uint8, (nb, d.page_size, d.latent_rank))
+        self._check("kv_rope", kv_rope, torch.bfloat16, (nb, d.page_size, d.rope_dim))
+        self._check("kv_scale", kv_scale, torch.float32, (nb, d.page_size))
         for name, t in (("q_nope", q_nope), ("q_rope", q_rope), ("kv_codes", kv_codes),
                         ("kv_rope", kv_rope), ("kv_scale", kv_scale), ("block_table", block_table),
                         ("seq_lens", seq_lens), ("w_uk", w_uk), ("w_uv", w_uv), ("out", out)):
             if not t.is_cuda or not t.is_contiguous():
                 raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if self.workspace is None:
+            self.allocate_workspace(q_nope.device)
         if stream is None:
             stream = torch.cuda.current_stream(q_nope.device).cuda_stream
         ev0, ev1 = (None, None) if decode_events is None else decode_events
