@@ -150,13 +150,18 @@ def test_split_partition_matches_independent_recomputation(seed):
         L.mla_plan_destroy(plan)
 
 
-def test_workspace_holds_partials_for_every_slot():
-    lens = [32768] * 32
+@pytest.mark.parametrize("batch", [32, 200000])
+def test_workspace_holds_partials_for_every_slot(batch):
+    # 200000 x 32K tokens: 1e8 pages and a workspace of ~100 GB, past every
+    # 32-bit count; the plan must size it without wrapping
+    lens = [32768] * batch
     plan, ws = L.mla_decode_plan_ex(_dims(), lens, num_sms=148, kernel=L.MLA_KERNEL_SIMT)
     try:
         info = L.mla_plan_get_info(plan)
         rows, slots = 128, info.num_split_slots
-        need = slots * rows * 512 * 4 + slots * rows * 4 + 32 * 128 * 576 * 2 + 33 * 8
+        assert slots == info.num_workers + batch - 1
+        assert info.total_pages == batch * 512
+        need = slots * rows * 512 * 4 + slots * rows * 4 + batch * 128 * 576 * 2 + (batch + 1) * 8
         assert ws >= need
     finally:
         L.mla_plan_destroy(plan)
