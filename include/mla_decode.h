@@ -184,7 +184,8 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan,
  * per group of 256 keys by a power of two into e4m3's normal range, as two
  * e4m3 terms; the result stays within twice the bf16 tolerance of the
  * dequantised cache. s_t must be positive and finite for every visible key
- * (any magnitude). */
+ * (any magnitude). The absorbed query q_nope . W_UK[h] must stay below 448 in
+ * magnitude (e4m3's largest finite value): larger entries saturate. */
 mla_status_t mla_decode_run_fp8(mla_plan_t plan,
                                 const void* q_nope, const void* q_rope,
                                 const void* kv_codes, const void* kv_rope, const float* kv_scale,
