@@ -170,8 +170,11 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan,
 
 /* One decode step over an FP8 latent cache (plan made with dims.dtype =
  * MLA_FP8_CACHE; mla_decode_run / _ex refuse such a plan with
- * MLA_ERR_INVALID_ARG). The cache is three device tensors over the same
- * blocks:
+ * MLA_ERR_INVALID_ARG). The operation is the one above on the dequantised
+ * cache; the TransMLA abstract names DeepSeek's FP8 quantisation among the
+ * optimisations a converted model can use, and this per-token-scale layout is
+ * this library's reading of it. The cache is three device tensors over the
+ * same blocks:
  *   kv_codes uint8 [num_blocks, page_size, r]   E4M3 ("e4m3fn") codes of cKV
  *   kv_rope  bf16  [num_blocks, page_size, d_rope] RoPE key divided by s_t
  *   kv_scale fp32  [num_blocks, page_size]      s_t, so that cKV_t = s_t * code_t
