@@ -45,7 +45,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="deepseek_v3")
-    ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05", "lsplit"], default="auto")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tcgen05"], default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="oracle work for the cpu_baseline sample")
@@ -419,7 +419,7 @@ def main():
     work = step_work(wl, lens)
     dev = {k: (v.to(device) if torch.is_tensor(v) else v) for k, v in inputs.items()}
     kernel = {"auto": M.MLA_KERNEL_AUTO, "simt": M.MLA_KERNEL_SIMT,
-              "tcgen05": M.MLA_KERNEL_TCGEN05, "lsplit": M.MLA_KERNEL_TCGEN05_LSPLIT}[args.kernel]
+              "tcgen05": M.MLA_KERNEL_TCGEN05}[args.kernel]
     dims = M.dims_for(wl.heads, wl.latent_rank, wl.rope_dim, wl.nope_dim, wl.v_dim, wl.q_len,
                       wl.softmax_scale, wl.dtype, wl.latent_shards, wl.page_size)
     plan = M.DecodePlan(dims, lens, kernel=kernel).allocate_workspace(device)
@@ -539,7 +539,7 @@ def main():
     value = whole_job_value(world, work["cache_bytes"], ms_step)
     e2e_value = whole_job_value(world, work["cache_bytes"], e2e_ms / Ke)
     info = plan.info
-    kname = {M.MLA_KERNEL_TCGEN05: "tcgen05", M.MLA_KERNEL_TCGEN05_LSPLIT: "tcgen05_lsplit"}.get(
+    kname = {M.MLA_KERNEL_TCGEN05: "tcgen05"}.get(
         info.kernel, "simt")
     dec_s = statistics.mean(decode_ms) * 1e-3
     hbm_peak = peaks["hbm_gbs"]

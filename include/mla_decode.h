@@ -14,7 +14,8 @@
  * results), "TransMLA: Multi-Head Latent Attention Is All You Need" abstract
  * (the Absorb operation keeps the cache compressed), the pith.science verdict
  * record for 2502.07864 (key_machinery: absorbed form is exact; core_discovery:
- * one shared multi-query RoPE key; referee report on Eq. 26: the MQA form).
+ * one RoPE key per token common to all heads; referee report on Eq. 26: the
+ * MQA form).
  *
  * Layouts (row-major, last dimension contiguous, element type = dims.dtype):
  *   q_nope   [B, Lq, H, d_nope]
@@ -79,9 +80,7 @@ typedef enum { MLA_BF16 = 0, MLA_FP32 = 1, MLA_FP8_CACHE = 2 } mla_dtype_t;
 typedef enum {
   MLA_KERNEL_AUTO = 0,    /* tcgen05 path where supported, else SIMT */
   MLA_KERNEL_SIMT = 1,    /* CUDA-core fp32 path (all dims; the fp32 path) */
-  MLA_KERNEL_TCGEN05 = 2, /* tensor-core path: bf16, r = 512, d_rope = 64, H*Lq <= 128 */
-  MLA_KERNEL_TCGEN05_LSPLIT = 3  /* tensor-core path whose CTA pairs split the cached columns
-                                    (each cached byte read once); one latent shard only */
+  MLA_KERNEL_TCGEN05 = 2  /* tensor-core path: bf16, r = 512, d_rope = 64, H*Lq <= 128 */
 } mla_kernel_t;
 
 typedef struct {
@@ -211,12 +210,19 @@ mla_status_t mla_decode_run_fp8(mla_plan_t plan,
  * fixed 32 MiB array in this library's device image (every GPU that loads the
  * library holds it until the process exits). Plans whose workspace_bytes
  * exceed 32 MiB are rejected with MLA_ERR_WORKSPACE_TOO_SMALL before any device
- * work; the DeepSeek-V3-shaped batch of 32 x 32K tokens on 148 SMs fits.
- * No cudaMalloc, cudaFree or other allocating call is made.
+ * work. On a 148-SM device the tensor-core plans of these batches fit: 16 x 8K
+ * tokens with 32 heads (~6.5 MB), 32 x 32K tokens with 128 heads, one or two
+ * latent shards (~32.3 MB); 64 sequences x 2 query tokens x 64 heads (~45 MB)
+ * do not. Plans over the FP8 cache are refused with MLA_ERR_UNSUPPORTED (this
+ * entry point wraps mla_decode_run only). No cudaMalloc, cudaFree or other
+ * allocating call is made.
  *
  * The first call on a device sets up that device: it resolves the array's
  * device address and clears its header (a synchronous memset followed by a
  * device synchronisation). Make that first call before any stream capture.
+ * The address is kept per device index for the life of the process: calls
+ * must run in the device's primary context (the CUDA runtime's), with no
+ * cudaDeviceReset in between.
  * All calls in the process share the one array per device and it keeps the
  * last call's contents; two calls whose work overlaps on the GPU (different
  * streams, or different threads) race on it and must be serialised by the

@@ -39,7 +39,6 @@ MLA_FP8_CACHE = 2
 MLA_KERNEL_AUTO = 0
 MLA_KERNEL_SIMT = 1
 MLA_KERNEL_TCGEN05 = 2
-MLA_KERNEL_TCGEN05_LSPLIT = 3
 
 # symbols declared in include/mla_decode.h
 EXPORTED = (

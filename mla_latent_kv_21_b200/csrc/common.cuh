@@ -130,6 +130,9 @@ struct RunParams {
   float scale_log2;        // softmax_scale * log2(e)
 };
 
+// True for a plan over the FP8 latent cache (host; defined with the ABI).
+bool plan_is_fp8(const mla_plan* plan);
+
 __device__ __forceinline__ void record_error(int32_t* status, int32_t code) {
   atomicCAS(status, 0, code);
 }

@@ -11,7 +11,6 @@
 #include "common.cuh"
 #include "simt_kernels.cuh"
 #include "tc_decode.cuh"
-#include "tc_decode_ls.cuh"
 #include "tc_decode_f8.cuh"
 #include "tc_head_gemm.cuh"
 
@@ -102,14 +101,11 @@ mla_status_t mla_decode_plan_ex(const mla_dims_t* dims, int32_t batch, const int
   if (dims->dtype == MLA_FP8_CACHE && (kernel != MLA_KERNEL_TCGEN05 || !tc_supported(*dims)))
     return MLA_ERR_UNSUPPORTED;
   if (kernel == MLA_KERNEL_TCGEN05 && !tc_supported(*dims)) return MLA_ERR_UNSUPPORTED;
-  if (kernel == MLA_KERNEL_TCGEN05_LSPLIT && !(tc_supported(*dims) && dims->latent_shards == 1))
-    return MLA_ERR_UNSUPPORTED;
-  if (kernel != MLA_KERNEL_SIMT && kernel != MLA_KERNEL_TCGEN05 && kernel != MLA_KERNEL_TCGEN05_LSPLIT)
-    return MLA_ERR_INVALID_ARG;
+  if (kernel != MLA_KERNEL_SIMT && kernel != MLA_KERNEL_TCGEN05) return MLA_ERR_INVALID_ARG;
   int64_t W;
   if (o.num_workers > 0) {
     W = o.num_workers;
-  } else if (kernel == MLA_KERNEL_TCGEN05 || kernel == MLA_KERNEL_TCGEN05_LSPLIT) {
+  } else if (kernel == MLA_KERNEL_TCGEN05) {
     // one CTA pair per worker (a cluster of two SMs); a pair step is one page
     W = std::max<int64_t>(1, std::min<int64_t>(sms / 2, G));
   } else {
@@ -141,6 +137,12 @@ mla_status_t mla_decode_plan(const mla_dims_t* dims, int32_t batch, const int32_
 }
 
 void mla_plan_destroy(mla_plan_t plan) { delete plan; }
+
+}  // extern "C"
+
+bool mla::plan_is_fp8(const mla_plan* plan) { return plan && plan->dims.dtype == MLA_FP8_CACHE; }
+
+extern "C" {
 
 mla_status_t mla_plan_get_info(mla_plan_t plan, mla_plan_info_t* info) {
   if (!plan || !info) return MLA_ERR_INVALID_ARG;
@@ -246,7 +248,7 @@ mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, c
 
   const bool bf16 = d.dtype == MLA_BF16;
   const int nbt = p.B * p.Lq;
-  const bool tc = plan->kernel == MLA_KERNEL_TCGEN05 || plan->kernel == MLA_KERNEL_TCGEN05_LSPLIT;
+  const bool tc = plan->kernel == MLA_KERNEL_TCGEN05;
   if (tc) {
     if (launch_absorb_tc(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
   } else {
@@ -263,8 +265,6 @@ mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, c
     if (launch_tc_decode_f8(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
   } else if (plan->kernel == MLA_KERNEL_TCGEN05) {
     if (launch_tc_decode(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
-  } else if (plan->kernel == MLA_KERNEL_TCGEN05_LSPLIT) {
-    if (launch_ls_decode(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
   } else {
     const size_t smem = simt_decode_smem_bytes(p.r + p.dr, p.S, p.P);
     const dim3 gd(p.W, (p.rows + kSimtRowGroup - 1) / kSimtRowGroup);

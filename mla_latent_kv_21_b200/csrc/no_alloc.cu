@@ -19,7 +19,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/mla_decode.h"
+#include "common.cuh"
 
 namespace {
 
@@ -31,18 +31,32 @@ static __device__ __align__(256) unsigned char mla_no_alloc_scratch[kNoAllocScra
 std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
 
+// A failed set-up step returns MLA_ERR_CUDA after taking its error off the
+// runtime's last-error slot, so that it does not surface later as the launch
+// error of an unrelated run.
+mla_status_t setup_failed() {
+  (void)cudaGetLastError();
+  return MLA_ERR_CUDA;
+}
+
 // Resolves (once per device) the device address of the scratch array and
-// clears its header so that the device status word starts at zero.
+// clears its header so that the device status word starts at zero. The
+// address is cached per device index for the life of the process, which
+// assumes the device's primary context (the one the CUDA runtime uses) and no
+// cudaDeviceReset between calls: a new context may place the array elsewhere.
 mla_status_t scratch_for_current_device(void** addr) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_NO_DEVICE;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MLA_ERR_NO_DEVICE;
+  }
   if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
   if (!g_scratch_addr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, mla_no_alloc_scratch) != cudaSuccess || !p) return MLA_ERR_CUDA;
-    if (cudaMemset(p, 0, 1024) != cudaSuccess) return MLA_ERR_CUDA;
-    if (cudaDeviceSynchronize() != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, mla_no_alloc_scratch) != cudaSuccess || !p) return setup_failed();
+    if (cudaMemset(p, 0, 1024) != cudaSuccess) return setup_failed();
+    if (cudaDeviceSynchronize() != cudaSuccess) return setup_failed();
     g_scratch_addr[dev] = p;
   }
   *addr = g_scratch_addr[dev];
@@ -61,6 +75,9 @@ extern "C" mla_status_t mla_decode_run_no_alloc(mla_plan_t plan, const void* q_n
   mla_plan_info_t info;
   mla_status_t st = mla_plan_get_info(plan, &info);
   if (st != MLA_OK) return st;
+  // the FP8 cache has its own entry point (mla_decode_run_fp8), which this one
+  // does not wrap
+  if (mla::plan_is_fp8(plan)) return MLA_ERR_UNSUPPORTED;
   // the plan's scratch must fit in the fixed array
   if (info.workspace_bytes > kNoAllocScratchBytes) return MLA_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;

@@ -39,7 +39,7 @@
 //
 // Sources: TPLA abstract (latent cache, shard-and-sum), TransMLA abstract
 // (absorbed decode over the compressed cache), pith.science verdict record for
-// 2502.07864 (shared multi-query RoPE key).
+// 2502.07864 (one RoPE key per token, common to all heads).
 #pragma once
 
 #include "common.cuh"

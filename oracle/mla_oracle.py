@@ -11,10 +11,11 @@ What it computes is the plain, non-absorbed definition of one MLA decode step
   a decoupled RoPE key shared by all heads (TPLA abstract, on the
   taxoreview listing pages; "TransMLA: Multi-Head Latent Attention Is All You
   Need", abstract; pith.science verdict record for 2502.07864, core_discovery:
-  "shared multi-query RoPE key").
+  one RoPE key per token, common to every head as in multi-query attention).
 * Per head h the keys and values are recovered through up-projections,
   K_h = [cKV . W_UK[h]^T || k_rope] and V_h = cKV . W_UV[h] (TransMLA v1
-  abstract on the kk6lht.com listing: MLA "employs an up-projection matrix").
+  abstract on the kk6lht.com listing: keys and values are recovered from the
+  latent by an up-projection).
   W_UK[h] is stored [d_nope, r] and W_UV[h] is stored [r, d_v].
 * Scores are scale * q . K_h[j] with q = [q_nope || q_rope]; query token t of
   Lq sees keys j <= L - Lq + t (the Lq query tokens are the newest Lq cache

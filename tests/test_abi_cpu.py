@@ -168,18 +168,14 @@ def test_workspace_holds_partials_for_every_slot(batch):
 
 
 @pytest.mark.parametrize("kw,kernel,status", [
-    # the latent-split kernel takes one latent shard, bf16
-    (dict(latent_shards=2), L.MLA_KERNEL_TCGEN05_LSPLIT, L.MLA_ERR_UNSUPPORTED),
     # the tensor-core kernels need r = 512 bf16; the fp32 tiny shape is SIMT only
     (dict(latent_rank=64, rope_dim=16, nope_dim=32, v_dim=32, dtype="fp32"),
      L.MLA_KERNEL_TCGEN05, L.MLA_ERR_UNSUPPORTED),
-    (dict(latent_rank=64, rope_dim=16, nope_dim=32, v_dim=32, dtype="fp32"),
-     L.MLA_KERNEL_TCGEN05_LSPLIT, L.MLA_ERR_UNSUPPORTED),
-    # unknown kernel kind
+    # unknown kernel kinds (3 was a removed latent-split variant)
+    (dict(), 3, L.MLA_ERR_INVALID_ARG),
     (dict(), 7, L.MLA_ERR_INVALID_ARG),
     # the FP8 cache runs on the tcgen05 decode kernel only, with one latent shard
     (dict(dtype="fp8"), L.MLA_KERNEL_SIMT, L.MLA_ERR_UNSUPPORTED),
-    (dict(dtype="fp8"), L.MLA_KERNEL_TCGEN05_LSPLIT, L.MLA_ERR_UNSUPPORTED),
     (dict(dtype="fp8", latent_shards=2), L.MLA_KERNEL_AUTO, L.MLA_ERR_UNSUPPORTED),
 ])
 def test_plan_rejects_unsupported_kernel_choices(kw, kernel, status):
@@ -188,8 +184,7 @@ def test_plan_rejects_unsupported_kernel_choices(kw, kernel, status):
     assert e.value.status == status
 
 
-@pytest.mark.parametrize("kernel", [L.MLA_KERNEL_AUTO, L.MLA_KERNEL_TCGEN05, L.MLA_KERNEL_TCGEN05_LSPLIT,
-                                    L.MLA_KERNEL_SIMT])
+@pytest.mark.parametrize("kernel", [L.MLA_KERNEL_AUTO, L.MLA_KERNEL_TCGEN05, L.MLA_KERNEL_SIMT])
 def test_plan_reports_kernel_and_launches(kernel):
     plan, ws = L.mla_decode_plan_ex(_dims(), [4000, 65], num_sms=148, kernel=kernel)
     try:
@@ -217,5 +212,44 @@ def test_fp8_plan_uses_tcgen05_and_bf16_run_refuses_it():
         with pytest.raises(L.MlaError) as e:
             L.mla_decode_run(plan, fake, fake, fake, 1, fake, 1, fake, fake, fake, fake, fake, ws, 0)
         assert e.value.status == L.MLA_ERR_INVALID_ARG
+    finally:
+        L.mla_plan_destroy(plan)
+
+
+def _kimi_lens():
+    from mla_workloads import WORKLOADS, draw_lengths
+    return draw_lengths(WORKLOADS["kimi_k2_mtp"]).tolist()
+
+
+@pytest.mark.parametrize("name,fits", [("tiny", True), ("llama2_7b", True), ("deepseek_v3", True),
+                                       ("tpla_dsv3", True), ("kimi_k2_mtp", False)])
+def test_no_alloc_scratch_covers_the_documented_plans(name, fits):
+    """The no-allocation entry point's fixed 32 MiB scratch holds the plans the
+    header lists (148 SMs, the default kernel) and refuses the larger one."""
+    from mla_workloads import WORKLOADS
+    wl = WORKLOADS[name]
+    lens = _kimi_lens() if wl.context_min else [wl.context] * wl.batch
+    dims = M.dims_for(wl.heads, wl.latent_rank, wl.rope_dim, wl.nope_dim, wl.v_dim, wl.q_len,
+                      wl.softmax_scale, wl.dtype, wl.latent_shards, wl.page_size)
+    plan, ws = L.mla_decode_plan(dims, lens, num_sms=148)
+    try:
+        assert (ws <= 32 << 20) == fits, ws
+        if not fits:
+            fake = 1 << 20  # never dereferenced: the size check comes before any device work
+            with pytest.raises(L.MlaError) as e:
+                L.mla_decode_run_no_alloc(plan, fake, fake, fake, 1, fake, 512, fake, fake, fake,
+                                          fake, 0)
+            assert e.value.status == L.MLA_ERR_WORKSPACE_TOO_SMALL
+    finally:
+        L.mla_plan_destroy(plan)
+
+
+def test_no_alloc_refuses_fp8_plans_before_any_device_work():
+    plan, _ = L.mla_decode_plan(_dims(dtype="fp8"), [4000, 65], num_sms=148)
+    try:
+        fake = 1 << 20  # never dereferenced: the dtype check comes before any device work
+        with pytest.raises(L.MlaError) as e:
+            L.mla_decode_run_no_alloc(plan, fake, fake, fake, 1, fake, 512, fake, fake, fake, fake, 0)
+        assert e.value.status == L.MLA_ERR_UNSUPPORTED
     finally:
         L.mla_plan_destroy(plan)

@@ -29,12 +29,7 @@ REDUCED = {
 }
 
 
-KERNELS = {"auto": M.MLA_KERNEL_AUTO, "simt": M.MLA_KERNEL_SIMT,
-           "lsplit": M.MLA_KERNEL_TCGEN05_LSPLIT}
-
-
-def _lsplit_ok(wl):
-    return wl.dtype == "bf16" and wl.latent_shards == 1
+KERNELS = {"auto": M.MLA_KERNEL_AUTO, "simt": M.MLA_KERNEL_SIMT}
 
 
 def _cases():
@@ -44,11 +39,9 @@ def _cases():
 
 
 @pytest.mark.parametrize("name,lens", list(_cases()))
-@pytest.mark.parametrize("kernel", ["auto", "simt", "lsplit"])
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
 def test_reduced_size_parity(cuda_device, name, lens, kernel):
     wl = WORKLOADS[name]
-    if kernel == "lsplit" and not _lsplit_ok(wl):
-        pytest.skip("the latent-split kernel takes bf16, one latent shard")
     k = KERNELS[kernel]
     inputs = generate(wl, seq_lens=lens)
     got, info = run_gpu(wl, inputs, cuda_device, kernel=k)
@@ -65,8 +58,7 @@ FULL_SAMPLES = {
 }
 
 
-@pytest.mark.parametrize("name,kernel", [(n, "auto") for n in FULL_SAMPLES]
-                         + [("deepseek_v3", "lsplit"), ("kimi_k2_mtp", "lsplit")])
+@pytest.mark.parametrize("name,kernel", [(n, "auto") for n in FULL_SAMPLES])
 def test_full_size_sampled_parity(cuda_device, name, kernel):
     wl = WORKLOADS[name]
     inputs = generate(wl)
