@@ -183,9 +183,10 @@ mla_status_t mla_decode_run_ex(mla_plan_t plan,
  * anything. Every other argument, the workspace and the errors are as for
  * mla_decode_run_ex. The tensor-core MMAs take e4m3 / e5m2 operands: the
  * absorbed query as an e4m3 value plus an e5m2 correction, and P * s_t, scaled
- * per group of 256 keys by a power of two into e4m3's normal range, as two
- * e4m3 terms; the result stays within twice the bf16 tolerance of the
- * dequantised cache. s_t must be positive and finite for every visible key
+ * per group of 256 keys by a power of two toward the top of e4m3's range, as
+ * two e4m3 terms; by the rounding steps alone the expected relative error
+ * against the dequantised cache (2.8e-3 rms) is below the bf16 path's
+ * (3.3e-3). s_t must be positive and finite for every visible key
  * (any magnitude). The absorbed query q_nope . W_UK[h] must stay below 448 in
  * magnitude (e4m3's largest finite value): larger entries saturate. */
 mla_status_t mla_decode_run_fp8(mla_plan_t plan,
@@ -236,6 +237,26 @@ mla_status_t mla_decode_run_no_alloc(mla_plan_t plan,
                                      const int32_t* seq_lens_dev,
                                      const void* w_uk, const void* w_uv,
                                      void* out, void* stream);
+
+/* Self-test of the device-side timeout path (diagnostics; not a decode).
+ * Runs one step of mla_decode_run on the same arguments, except that in the
+ * split-KV decode kernel every bounded wait gives up after wait_limit_ns
+ * (1 us .. 2 s) instead of 2 s, and the softmax warps withhold the release of
+ * their score buffers in tensor memory. A worker with three or more groups of
+ * 256 keys then reaches a wait that nothing completes: that wait runs out, the
+ * kernel records MLA_ERR_DEVICE_TIMEOUT in the workspace status word, its
+ * other roles stop at their next wait, the tensor memory is released and the
+ * kernel returns; no trap, fault or hang, and the context stays usable. The
+ * output is undefined. Read the status with mla_decode_read_status. Plans for
+ * the bf16 cache on the tensor-core kernel only (else MLA_ERR_UNSUPPORTED). */
+mla_status_t mla_decode_selftest_timeout(mla_plan_t plan,
+                                         const void* q_nope, const void* q_rope,
+                                         const void* kv_cache, int64_t num_blocks,
+                                         const int32_t* block_table, int32_t block_table_stride,
+                                         const int32_t* seq_lens_dev,
+                                         const void* w_uk, const void* w_uv,
+                                         void* out, void* workspace, size_t workspace_bytes,
+                                         uint64_t wait_limit_ns, void* stream);
 
 /* Clears the workspace header (status word) with an async memset on `stream`.
  * Call once after allocating a workspace, before its first run. */

@@ -43,7 +43,7 @@ MLA_KERNEL_TCGEN05 = 2
 # symbols declared in include/mla_decode.h
 EXPORTED = (
     "mla_decode_plan", "mla_decode_plan_ex", "mla_decode_run", "mla_decode_run_ex",
-    "mla_decode_run_fp8", "mla_decode_run_no_alloc", "mla_workspace_init",
+    "mla_decode_run_fp8", "mla_decode_run_no_alloc", "mla_decode_selftest_timeout", "mla_workspace_init",
     "mla_decode_read_status", "mla_plan_get_info", "mla_plan_segments", "mla_plan_destroy",
     "mla_status_string", "mla_abi_version",
 )
@@ -99,6 +99,9 @@ _lib.mla_decode_run_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _i3
 _lib.mla_decode_run_no_alloc.restype = ctypes.c_int
 _lib.mla_decode_run_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp,
                                          _vp]
+_lib.mla_decode_selftest_timeout.restype = ctypes.c_int
+_lib.mla_decode_selftest_timeout.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp,
+                                             _vp, _sz, ctypes.c_uint64, _vp]
 _lib.mla_workspace_init.restype = ctypes.c_int
 _lib.mla_workspace_init.argtypes = [_vp, _sz, _vp]
 _lib.mla_decode_read_status.restype = ctypes.c_int
@@ -198,6 +201,17 @@ def mla_decode_run_no_alloc(plan, q_nope, q_rope, kv_cache, num_blocks, block_ta
     _check(_lib.mla_decode_run_no_alloc(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,
                                         block_table_stride, seq_lens_dev, w_uk, w_uv, out,
                                         stream), "mla_decode_run_no_alloc")
+
+
+def mla_decode_selftest_timeout(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,
+                                block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace,
+                                workspace_bytes, wait_limit_ns, stream=0) -> None:
+    """Diagnostics: a decode step whose decode kernel withholds one barrier
+    arrival with every wait bounded by wait_limit_ns (see the C header)."""
+    _check(_lib.mla_decode_selftest_timeout(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,
+                                            block_table_stride, seq_lens_dev, w_uk, w_uv, out,
+                                            workspace, workspace_bytes, wait_limit_ns, stream),
+           "mla_decode_selftest_timeout")
 
 
 def mla_workspace_init(workspace, workspace_bytes, stream=0) -> None:

@@ -128,6 +128,11 @@ struct RunParams {
   int32_t W;               // workers
   int32_t fp8;             // 1: FP8 cache (the absorbed query is written as e4m3 + e5m2 bytes)
   float scale_log2;        // softmax_scale * log2(e)
+  // bounded waits of the bf16 tensor-core decode kernel (2 s in a normal run)
+  uint64_t wait_limit_ns;
+  // self-test of the timeout path only: the decode kernel's softmax withholds
+  // the release of its score buffers, so the QK issuer's wait runs out
+  int32_t withhold_s_free;
 };
 
 // True for a plan over the FP8 latent cache (host; defined with the ABI).

@@ -200,11 +200,18 @@ mla_status_t mla_decode_run(mla_plan_t plan, const void* q_nope, const void* q_r
 
 namespace {
 
+// Device-wait settings of one run: the normal limit, or a self-test of the
+// timeout path (short limit, one arrival withheld in the decode kernel).
+struct WaitKnobs {
+  uint64_t limit_ns = ptx::kWaitLimitNs;
+  int32_t withhold_s_free = 0;
+};
+
 mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, const void* kv_cache,
                       const void* kv_rope, const float* kv_scale, int64_t num_blocks,
                       const int32_t* block_table, int32_t block_table_stride, const int32_t* seq_lens_dev,
                       const void* w_uk, const void* w_uv, void* out, void* workspace, size_t workspace_bytes,
-                      void* stream_, const mla_run_options_t* opts) {
+                      void* stream_, const mla_run_options_t* opts, WaitKnobs knobs = WaitKnobs{}) {
   if (!plan || !q_nope || !q_rope || !kv_cache || !block_table || !seq_lens_dev || !w_uk ||
       !w_uv || !out || !workspace || num_blocks < 1 || block_table_stride < 1)
     return MLA_ERR_INVALID_ARG;
@@ -245,6 +252,8 @@ mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, c
   p.rows = d.num_heads * d.q_len;
   p.W = plan->W;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  p.wait_limit_ns = knobs.limit_ns;
+  p.withhold_s_free = knobs.withhold_s_free;
 
   const bool bf16 = d.dtype == MLA_BF16;
   const int nbt = p.B * p.Lq;
@@ -319,6 +328,23 @@ mla_status_t mla_decode_run_fp8(mla_plan_t plan, const void* q_nope, const void*
   if (!plan || plan->dims.dtype != MLA_FP8_CACHE || !kv_rope || !kv_scale) return MLA_ERR_INVALID_ARG;
   return run_impl(plan, q_nope, q_rope, kv_codes, kv_rope, kv_scale, num_blocks, block_table,
                   block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace, workspace_bytes, stream_, opts);
+}
+
+mla_status_t mla_decode_selftest_timeout(mla_plan_t plan, const void* q_nope, const void* q_rope,
+                                         const void* kv_cache, int64_t num_blocks,
+                                         const int32_t* block_table, int32_t block_table_stride,
+                                         const int32_t* seq_lens_dev, const void* w_uk, const void* w_uv,
+                                         void* out, void* workspace, size_t workspace_bytes,
+                                         uint64_t wait_limit_ns, void* stream_) {
+  // the bf16 tensor-core decode kernel is the one whose waits take the limit
+  if (!plan || plan->dims.dtype != MLA_BF16 || plan->kernel != MLA_KERNEL_TCGEN05) return MLA_ERR_UNSUPPORTED;
+  if (wait_limit_ns < 1000 || wait_limit_ns > ptx::kWaitLimitNs) return MLA_ERR_INVALID_ARG;
+  WaitKnobs k;
+  k.limit_ns = wait_limit_ns;
+  k.withhold_s_free = 1;
+  return run_impl(plan, q_nope, q_rope, kv_cache, nullptr, nullptr, num_blocks, block_table,
+                  block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace, workspace_bytes, stream_,
+                  nullptr, k);
 }
 
 mla_status_t mla_workspace_init(void* workspace, size_t workspace_bytes, void* stream_) {

@@ -2,9 +2,9 @@
 // mbarriers (with bounded waits), TMA tile loads, tensor-memory allocation,
 // tcgen05 MMA / commit / load / store, and cluster (CTA-pair) helpers.
 //
-// Every wait in this file is bounded: after kWaitLimitNs of wall time it gives
-// up and returns false so the caller can record MLA_ERR_DEVICE_TIMEOUT and
-// unwind instead of hanging the GPU.
+// Every wait in this file is bounded: after kWaitLimitNs (or the caller's
+// limit) of wall time it gives up and returns false so the caller can record
+// MLA_ERR_DEVICE_TIMEOUT and unwind instead of hanging the GPU.
 #pragma once
 
 #include <cstdint>
@@ -119,18 +119,19 @@ __device__ __forceinline__ bool mbar_try_wait_cta(uint32_t bar, uint32_t parity)
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete. kCluster
-// selects a cluster-scope acquire; the kernels use the CTA-scope form (the
-// cluster-scope one costs throughput next to in-flight TMA loads, and the
-// peer's arrivals publish nothing that this CTA's threads read).
+// Bounded wait for the phase with the given parity to complete: false once
+// limit_ns of wall time have passed. kCluster selects a cluster-scope acquire;
+// the kernels use the CTA-scope form (the cluster-scope one costs throughput
+// next to in-flight TMA loads, and the peer's arrivals publish nothing that
+// this CTA's threads read).
 template <bool kCluster = false>
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   auto probe = [&]() { return kCluster ? mbar_try_wait(bar, parity) : mbar_try_wait_cta(bar, parity); };
   if (probe()) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (probe()) return true;
-    if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if ((it & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 

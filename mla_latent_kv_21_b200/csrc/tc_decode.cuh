@@ -320,7 +320,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kc = 0; kc < kChunks && ok; ++kc, ++cc) {
           const int slot = cc % C::kQkSlots;
           if (cc >= (uint32_t)C::kQkSlots)
-            ok = mbar_wait(bar(B_QK_FREE + slot), ((cc / C::kQkSlots) - 1) & 1);
+            ok = mbar_wait(bar(B_QK_FREE + slot), ((cc / C::kQkSlots) - 1) & 1, p.wait_limit_ns);
           if (!ok) break;
           if (g.first && lane == 1) {
             // New segment: reload query chunk kc. Its last reader, chunk kc of
@@ -355,7 +355,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int nb = 0; nb < 2 && ok; ++nb, ++vc) {
             const int slot = vc % C::kVSlots;
             if (vc >= (uint32_t)C::kVSlots)
-              ok = mbar_wait(bar(B_V_FREE + slot), ((vc / C::kVSlots) - 1) & 1);
+              ok = mbar_wait(bar(B_V_FREE + slot), ((vc / C::kVSlots) - 1) & 1, p.wait_limit_ns);
             if (!ok) break;
             if (lane == 0) expect_leader(B_V_FULL + slot, kSlotBytes);
             const int chunk = 4 * nb + 2 * (int)rank + lane;
@@ -383,14 +383,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool have = g.init(p, w);
       for (int gi = 0; have && ok; ++gi) {
         const int sb = gi % C::kSBufs;
-        if (ok && gi >= C::kSBufs) ok = mbar_wait(bar(B_S_FREE + sb), ((gi / C::kSBufs) - 1) & 1);
+        if (ok && gi >= C::kSBufs) ok = mbar_wait(bar(B_S_FREE + sb), ((gi / C::kSBufs) - 1) & 1, p.wait_limit_ns);
         if (!ok) break;
         MLA_TRACE_EV(w, 0, EV_QK_START, gi);
         const uint32_t s_tmem = tbase + sb * 128 * S;
         for (int kc = 0; kc < kChunks && ok; ++kc, ++cc) {
           const int slot = cc % C::kQkSlots;
-          if (g.first) ok = mbar_wait(bar(B_QC_FULL + kc), g.seg & 1);  // this segment's query chunk
-          ok = ok && mbar_wait(bar(B_QK_FULL + slot), (cc / C::kQkSlots) & 1);
+          if (g.first) ok = mbar_wait(bar(B_QC_FULL + kc), g.seg & 1, p.wait_limit_ns);  // this segment's query chunk
+          ok = ok && mbar_wait(bar(B_QK_FULL + slot), (cc / C::kQkSlots) & 1, p.wait_limit_ns);
           if (!ok) break;
           MLA_TRACE_CHUNK(w, 0, 1, cc);
           tc_fence_after();
@@ -413,7 +413,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         have = g.next(p);
       }
       tc_commit<2>(bar(B_FINAL_QK));
-      if (!mbar_wait(bar(B_FINAL_QK), 0)) ok = false;
+      if (!mbar_wait(bar(B_FINAL_QK), 0, p.wait_limit_ns)) ok = false;
       if (!ok) fail(MLA_ERR_DEVICE_TIMEOUT);
     }
     __syncwarp();
@@ -428,20 +428,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       GroupCursor g;
       bool have = g.init(p, w);
       for (int gi = 0; have && ok; ++gi) {
-        ok = mbar_wait(bar(B_P_FULL), gi & 1);
-        if (ok && g.first && g.seg > 0) ok = mbar_wait(bar(B_O_FREE), (g.seg - 1) & 1);
+        ok = mbar_wait(bar(B_P_FULL), gi & 1, p.wait_limit_ns);
+        if (ok && g.first && g.seg > 0) ok = mbar_wait(bar(B_O_FREE), (g.seg - 1) & 1, p.wait_limit_ns);
         if (!ok) break;
         MLA_TRACE_EV(w, 0, EV_PV_START, gi);
         // page-major: P of pages 0, 1 is released half way through
         for (int q = 0; q < kGroupPages && ok; ++q) {
           if (C::kSharedP && q == 2) {
-            ok = mbar_wait(bar(B_P_FULL_HI), gi & 1);  // pages 2, 3 in the shared P buffer
+            ok = mbar_wait(bar(B_P_FULL_HI), gi & 1, p.wait_limit_ns);  // pages 2, 3 in the shared P buffer
             if (!ok) break;
           }
           for (int nb = 0; nb < 2 && ok; ++nb, ++vc) {
             const int shard = S == 2 ? nb : 0;
             const int slot = vc % C::kVSlots;
-            ok = mbar_wait(bar(B_V_FULL + slot), (vc / C::kVSlots) & 1);
+            ok = mbar_wait(bar(B_V_FULL + slot), (vc / C::kVSlots) & 1, p.wait_limit_ns);
             if (!ok) break;
             MLA_TRACE_CHUNK(w, 0, 3, vc);
             tc_fence_after();
@@ -464,7 +464,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         have = g.next(p);
       }
       tc_commit<2>(bar(B_FINAL_PV));
-      if (!mbar_wait(bar(B_FINAL_PV), 0)) ok = false;
+      if (!mbar_wait(bar(B_FINAL_PV), 0, p.wait_limit_ns)) ok = false;
       if (!ok) fail(MLA_ERR_DEVICE_TIMEOUT);
     }
     __syncwarp();
@@ -485,7 +485,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto named_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
     auto wait = [&](int b, uint32_t parity) {
       if (ok && *abort_flag) ok = false;
-      if (ok) ok = mbar_wait(bar(b), parity);
+      if (ok) ok = mbar_wait(bar(b), parity, p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);
     };
     GroupCursor g;
@@ -529,7 +529,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // every score of this S buffer is in registers: QK may reuse it
           if (ok) tc_fence_before();
           __syncwarp();
-          if (ok && lane == 0) arrive_leader(B_S_FREE + sb);
+          if (ok && lane == 0 && !p.withhold_s_free) arrive_leader(B_S_FREE + sb);
         }
         // masked keys (past the group or the causal limit) become -inf: they
         // drop out of the max and 2^-inf = 0 in the sum and in P

@@ -24,9 +24,11 @@
 //       P'_lo = e4m3(P' - P'_hi) and each K step of 32 tokens takes two
 //       kind::f8f6f4 MMAs (P'_hi . code and P'_lo . code), so O accumulates
 //       2^kp sum_t p_t cKV_t. The power of two 2^kp, chosen per group from the
-//       group's largest scale, puts the largest weights near 1 (in e4m3's
-//       normal range) and is carried by O and the row sum like a shift of
-//       the running max.
+//       group's largest scale, puts P' as high in e4m3's range as the lazy max
+//       allows (28 < 2^kp * s_max <= 56 and P <= 2^3: P' <= 448), so that
+//       every weight P >= (s_max / s_t) / 112 has P' >= 1/4, where the split
+//       keeps 8 significant bits; it is carried by O and the row sum like a
+//       shift of the running max.
 //   softmax  the per-element work is about three times the bf16 kernel's, so
 //       both passes (row max; P, P' and its split) walk a thread's 128 columns
 //       32 at a time through one copy of their loop body, reading S from
@@ -38,8 +40,8 @@
 // The two-term splits keep the operands near bf16 precision while the cache
 // bytes per token fall from 1152 to 644: the e4m3 term leaves a residual below
 // 2^-4 of the value, which the query's e5m2 term (any magnitude) carries to
-// within 2^-3 of itself and P's e4m3 term (P' near 1) to within 2^-4, or to an
-// absolute 2^-10 when the residual is below e4m3's normal range.
+// within 2^-3 of itself and P's e4m3 term to within 2^-4 while the residual is
+// an e4m3 normal (P' >= 1/4), or to an absolute 2^-10 below that.
 //
 // Sources: as tc_decode.cuh (TPLA abstract, TransMLA abstract, pith.science
 // verdict record for 2502.07864); the FP8 cache itself is a format of this
@@ -55,7 +57,11 @@ namespace tc8 {
 
 using tc::GroupCursor;
 using tc::kGroupPages;
-using tc::kRescaleThreshold;
+// The running max moves (and O is rescaled) when a group's row max exceeds it
+// by more than 2^3, so P <= 2^3 and P' = 2^kp * P * s_t <= 8 * kPScaleTarget
+// = 448, e4m3's largest finite value.
+constexpr float kRescaleThreshold = 3.0f;   // log2 units
+constexpr float kPScaleTarget = 56.0f;      // 2^kp * s_max <= 56
 using tc::kThreads;
 using tc::kTmemCols;
 using tc::kTmemO;
@@ -543,13 +549,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float mt = fmaxf(mt_own, xmax[lq ^ 64]);
       float mu = m;
       if (m == -INFINITY || mt > m + kRescaleThreshold) mu = fmaxf(mt, m);
-      // P' is kept as 2^kp * P * s_t with 2^kp * s_max <= 1.75, so that with
-      // P <= 2^8 (the lazy max) it stays below e4m3's 448 and the group's
-      // largest weights sit near 1, in e4m3's normal range; kp only falls
-      // within a segment. O and l carry the same 2^kp: the exponent offset is
-      // m - kp, and a change of either rescales them like a new max.
+      // P' is kept as 2^kp * P * s_t with 2^kp * s_max <= 56, so that with
+      // P <= 2^3 (the lazy max) it stays at or below e4m3's 448 and weights
+      // P >= (s_max / s_t) / 112 reach P' >= 1/4 (8 bits in the split); kp
+      // only falls within a segment. O and l carry the same 2^kp: the exponent
+      // offset is m - kp, and a change of either rescales them like a new max.
       const float smax = fmaxf(fmaxf(xsmax[0], xsmax[1]), fmaxf(xsmax[2], xsmax[3]));
-      int kg = smax > 0.f ? (int)((__float_as_uint(1.75f / smax) >> 23) & 0xFF) - 127 : kp;
+      int kg = smax > 0.f ? (int)((__float_as_uint(kPScaleTarget / smax) >> 23) & 0xFF) - 127 : kp;
       kg = kg < -64 ? -64 : (kg > 64 ? 64 : kg);
       const int kn = g.first ? kg : min(kp, kg);
       const float off_old = m - (float)kp, off_new = mu - (float)kn;

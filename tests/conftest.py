@@ -18,3 +18,20 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+_PARITY_REPORT = []
+
+
+@pytest.fixture(scope="session")
+def parity_report():
+    """Tests append (workload, what, max_abs, rel_fro); the terminal summary
+    prints them, so the figures appear in a quiet run's output too."""
+    return _PARITY_REPORT
+
+
+def pytest_terminal_summary(terminalreporter):
+    if _PARITY_REPORT:
+        terminalreporter.write_sep("-", "full-size parity against the oracle")
+        for name, what, max_abs, rel in _PARITY_REPORT:
+            terminalreporter.write_line(f"{name}: {what}: max_abs {max_abs:.3e} rel_fro {rel:.3e}")

@@ -253,3 +253,23 @@ def test_no_alloc_refuses_fp8_plans_before_any_device_work():
         assert e.value.status == L.MLA_ERR_UNSUPPORTED
     finally:
         L.mla_plan_destroy(plan)
+
+
+@pytest.mark.parametrize("kw,kernel,limit,status", [
+    (dict(), L.MLA_KERNEL_SIMT, 1_000_000, L.MLA_ERR_UNSUPPORTED),
+    (dict(dtype="fp8"), L.MLA_KERNEL_TCGEN05, 1_000_000, L.MLA_ERR_UNSUPPORTED),
+    (dict(), L.MLA_KERNEL_TCGEN05, 999, L.MLA_ERR_INVALID_ARG),
+    (dict(), L.MLA_KERNEL_TCGEN05, 3_000_000_000, L.MLA_ERR_INVALID_ARG),
+])
+def test_timeout_selftest_argument_checks(kw, kernel, limit, status):
+    """The timeout self-test takes bf16 tensor-core plans and a limit in
+    [1 us, 2 s]; the checks come before any device work."""
+    plan, ws = L.mla_decode_plan_ex(_dims(**kw), [4000, 65], num_sms=148, kernel=kernel)
+    try:
+        fake = 1 << 20  # never dereferenced
+        with pytest.raises(L.MlaError) as e:
+            L.mla_decode_selftest_timeout(plan, fake, fake, fake, 1, fake, 64, fake, fake, fake, fake,
+                                          fake, ws, limit, 0)
+        assert e.value.status == status
+    finally:
+        L.mla_plan_destroy(plan)

@@ -8,7 +8,6 @@ e4m3 terms, the fp16 partials, bf16 output) against the FP8 tolerance.
 
 import dataclasses
 
-import numpy as np
 import pytest
 import torch
 
@@ -35,16 +34,6 @@ def test_split_counts(cuda_device, workers):
     inputs = generate(WL, seq_lens=[1200, 70, 3])
     got, info = run_gpu(WL, inputs, cuda_device, num_workers=workers)
     assert_close(got.double().numpy(), oracle_out(WL, inputs), WL.dtype, f"workers={info.num_workers}")
-
-
-def test_full_size_sampled_parity(cuda_device):
-    inputs = generate(WL)
-    got, _ = run_gpu(WL, inputs, cuda_device)
-    got = got.double().numpy()
-    assert np.isfinite(got).all()
-    for b, h in [(0, 0), (13, 77), (31, 127)]:
-        ref = oracle_out(WL, inputs, [b], [h])[0, :, 0]
-        assert_close(got[b, :, h], ref, WL.dtype, f"b={b} h={h}")
 
 
 @pytest.mark.parametrize("lens", [[2, 65, 300, 1030], [129, 3]])

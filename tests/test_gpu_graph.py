@@ -8,14 +8,13 @@ reproduce the eager output bit for bit (the decode is deterministic) and stay
 within the oracle tolerance.
 """
 
-import numpy as np
 import pytest
 import torch
 
 import mla_latent_kv_21_b200 as M
 from mla_workloads import WORKLOADS, generate
 
-from harness import TOL, dims_of, errors, oracle_out, to_device
+from harness import assert_close, dims_of, oracle_out, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -59,8 +58,6 @@ def test_graph_replay_matches_eager(cuda_device, name, lens):
         assert torch.equal(out, eager), "graph replay differs from the eager run"
     got = out.double().cpu().numpy()
     ref = oracle_out(wl, inputs)
-    max_abs, rel = errors(got, ref)
-    tol = TOL[wl.dtype]
-    assert rel <= tol["rel_fro"] and (wl.dtype != "bf16" or max_abs <= tol["max_abs"])
+    assert_close(got, ref, wl.dtype, f"{wl.name} graph replay")
     del g
     plan.close()
