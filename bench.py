@@ -49,6 +49,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="oracle work for the cpu_baseline sample")
+    ap.add_argument("--tpla-shard", action="store_true",
+                    help="TPLA workloads on one GPU: time one GPU's latent shard of the multi-GPU form "
+                         "(no all-reduce: the other shards live on other GPUs)")
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling cases)")
     ap.add_argument("--context", type=int, default=0, help="override every length (profiling cases)")
     return ap.parse_args()
@@ -282,6 +285,17 @@ def max_over_ranks(x: float, dist, device) -> float:
     return float(t.item())
 
 
+def tpla_layout(world: int, tp: int) -> dict:
+    """Ranks of a TPLA run across GPUs: consecutive groups of tp ranks (one
+    latent shard per rank, an all-reduce inside each group), the groups
+    decoding independent replicas of the batch."""
+    if tp < 1 or world % tp:
+        raise ValueError(f"{world} ranks do not split into groups of {tp}")
+    groups = [list(range(i, i + tp)) for i in range(0, world, tp)]
+    return {"groups": groups, "tp_rank": [r % tp for r in range(world)],
+            "group_of": [r // tp for r in range(world)]}
+
+
 def whole_job_value(world: int, bytes_per_rank: float, ms_per_step: float) -> float:
     """GB/s of the whole job: every rank processes its own full batch (weak
     scaling, replicas), timed by the slowest rank."""
@@ -419,13 +433,31 @@ def main():
 
     inputs = generate(wl)
     lens = inputs["seq_lens"].tolist()
-    work = step_work(wl, lens)
-    dev = {k: (v.to(device) if torch.is_tensor(v) else v) for k, v in inputs.items()}
     kernel = {"auto": M.MLA_KERNEL_AUTO, "simt": M.MLA_KERNEL_SIMT,
               "tcgen05": M.MLA_KERNEL_TCGEN05}[args.kernel]
     dims = M.dims_for(wl.heads, wl.latent_rank, wl.rope_dim, wl.nope_dim, wl.v_dim, wl.q_len,
                       wl.softmax_scale, wl.dtype, wl.latent_shards, wl.page_size)
-    plan = M.DecodePlan(dims, lens, kernel=kernel).allocate_workspace(device)
+    # TPLA on more than one GPU: groups of latent_shards ranks, one latent shard
+    # per rank, the shard outputs summed by one all-reduce per step (the
+    # method's exchange step); every other workload runs replicas
+    tp = wl.latent_shards if ((dist or args.tpla_shard) and wl.latent_shards > 1) else 1
+    if tp > 1:
+        from mla_workloads import tpla_shard_inputs
+        if dist:
+            lay = tpla_layout(world, tp)
+            groups = [dist.new_group(g) for g in lay["groups"]]
+            tp_rank, group = lay["tp_rank"][rank], groups[lay["group_of"][rank]]
+        else:
+            tp_rank, group = 0, None
+        inputs = tpla_shard_inputs(inputs, wl, tp, tp_rank)
+        plan = M.TplaShardPlan(dims, lens, tp=tp, group=group).allocate_workspace(device)
+        if not dist:
+            plan.run = plan.run_shard  # one GPU holds one shard here: nothing to sum
+        work = step_work(wl.with_(latent_rank=wl.latent_rank // tp, latent_shards=1), lens)
+    else:
+        plan = M.DecodePlan(dims, lens, kernel=kernel).allocate_workspace(device)
+        work = step_work(wl, lens)
+    dev = {k: (v.to(device) if torch.is_tensor(v) else v) for k, v in inputs.items()}
     B = len(lens)
     out = torch.empty((B, wl.q_len, wl.heads, wl.v_dim), dtype=wl.torch_dtype, device=device)
     stream = torch.cuda.current_stream(device)
@@ -587,7 +619,10 @@ def main():
                    "rope_dim": wl.rope_dim, "nope_dim": wl.nope_dim, "v_dim": wl.v_dim,
                    "latent_shards": wl.latent_shards, "page_size": wl.page_size,
                    "kernel": kname, "workers": info.num_workers,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "parallelism": (f"tpla: {world // tp} groups x {tp} latent shards, all-reduce"
+                                   if tp > 1 and dist else
+                                   f"one latent shard of {tp} (the per-GPU work of TPLA across GPUs)"
+                                   if tp > 1 else f"replicas{world}" if world > 1 else "single"),
                    "l2": f"inputs larger than L2 (cache {work['cache_bytes'] / 1e9:.2f} GB)"},
         "us_per_step": ms_step * 1e3,
         "tflops": work["step_flops"] / (ms_step * 1e-3) / 1e12,
@@ -601,7 +636,7 @@ def main():
         "clocks": sampler.summary(w0, w_head),
     }
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and tp == 1 and not args.no_cpu_baseline:
         # the oracle as it stands on the host cores, bounded sample; its sampled
         # outputs double as a parity spot check of this run's GPU output
         # seeded (sequence, head) pairs at full length until about

@@ -80,7 +80,9 @@ typedef enum { MLA_BF16 = 0, MLA_FP32 = 1, MLA_FP8_CACHE = 2 } mla_dtype_t;
 typedef enum {
   MLA_KERNEL_AUTO = 0,    /* tcgen05 path where supported, else SIMT */
   MLA_KERNEL_SIMT = 1,    /* CUDA-core fp32 path (all dims; the fp32 path) */
-  MLA_KERNEL_TCGEN05 = 2  /* tensor-core path: bf16, r = 512, d_rope = 64, H*Lq <= 128 */
+  MLA_KERNEL_TCGEN05 = 2  /* tensor-core path: d_rope = 64, d_nope = d_v = 128, H*Lq <= 128;
+                             bf16 with r = 512 (1 or 2 latent shards) or r = 256 (1 shard:
+                             one TPLA shard per GPU), or the FP8 cache with r = 512 */
 } mla_kernel_t;
 
 typedef struct {

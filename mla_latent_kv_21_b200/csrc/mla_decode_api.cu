@@ -29,10 +29,16 @@ struct mla_plan {
 
 namespace {
 
+// The tensor-core kernels: r = 512 (bf16 with one or two latent shards, or the
+// FP8 cache), or r = 256 with one shard (bf16; a TPLA shard per GPU).
 bool tc_supported(const mla_dims_t& d) {
-  return kTcDecodeAvailable && (d.dtype == MLA_BF16 || d.dtype == MLA_FP8_CACHE) && d.latent_rank == 512 &&
-         d.rope_dim == 64 && d.page_size == 64 && d.num_heads * d.q_len <= 128 && d.nope_dim == 128 &&
-         d.v_dim == 128 && (d.latent_shards == 1 || (d.latent_shards == 2 && d.dtype == MLA_BF16));
+  if (!(kTcDecodeAvailable && d.rope_dim == 64 && d.page_size == 64 && d.num_heads * d.q_len <= 128 &&
+        d.nope_dim == 128 && d.v_dim == 128))
+    return false;
+  if (d.latent_rank == 512)
+    return d.dtype == MLA_BF16 ? (d.latent_shards == 1 || d.latent_shards == 2)
+                               : (d.dtype == MLA_FP8_CACHE && d.latent_shards == 1);
+  return d.latent_rank == 256 && d.dtype == MLA_BF16 && d.latent_shards == 1;
 }
 
 mla_status_t check_dims(const mla_dims_t& d) {

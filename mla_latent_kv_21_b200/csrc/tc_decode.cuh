@@ -51,13 +51,25 @@ constexpr bool kTcDecodeAvailable = true;
 
 namespace tc {
 
-constexpr int kWidth = 576;                 // r + d_rope
-constexpr int kChunks = 9;                  // 64-column chunks of a row (8 latent + 1 rope)
+constexpr int kWidth = 576;                 // r + d_rope at r = 512
+constexpr int kChunks = 9;                  // 64-column chunks of a row at r = 512 (8 latent + 1 rope)
 constexpr int kGroupPages = 4;              // pages per pair step (256 tokens)
 // warps: 0 Q/QK loads, 1 QK MMA, 2 V loads, 3-6 softmax, 7 PV MMA
 constexpr int kThreads = 256;
 constexpr uint32_t kQChunkBytes = 64 * 128;  // 64 rows x 128 B
 constexpr uint32_t kQBytes = kChunks * kQChunkBytes;
+// The latent width R of one launch: 512 (every workload on one GPU), or 256
+// (one latent shard per GPU of a tensor-parallel pair: TPLA across GPUs).
+// Per R: 64-column chunks of a cached row (latent + RoPE), PV N blocks of 256
+// latent columns, and the tensor-memory columns of this CTA's O accumulator.
+template <int R>
+struct Width {
+  static_assert(R == 256 || R == 512, "latent width 256 or 512");
+  static constexpr int kChunks = R / 64 + 1;
+  static constexpr int kNBlocks = R / 256;
+  static constexpr uint32_t kQBytes = kChunks * kQChunkBytes;
+  static constexpr uint32_t kOCols = R / 2;
+};
 constexpr uint32_t kSlotBytes = 16384;       // QK slot: 128 tokens x 64 cols; V slot: 64 tokens x 128 cols
 constexpr uint32_t kPChunkBytes = 64 * 128;  // 64 rows x 64 tokens bf16
 constexpr uint32_t kPBytes = 4 * kPChunkBytes;  // 64 rows x 256 tokens
@@ -75,7 +87,7 @@ constexpr int kIssueLanes = 2;
 #ifndef MLA_V_SLOTS
 #define MLA_V_SLOTS 4
 #endif
-template <int S>
+template <int S, int R = 512>
 struct Cfg {
   static constexpr int kQkSlots = S == 1 ? MLA_QK_SLOTS : 3;
   static constexpr int kVSlots = S == 1 ? MLA_V_SLOTS : 2;
@@ -87,18 +99,18 @@ struct Cfg {
   static constexpr uint32_t kPRegion = kSharedP ? kPBytes / 2 : S * kPBytes;
 };
 
-template <int S>
+template <int S, int R = 512>
 struct Smem {
   static constexpr uint32_t q = 0;
-  static constexpr uint32_t qk = q + kQBytes;
-  static constexpr uint32_t v = qk + Cfg<S>::kQkSlots * kSlotBytes;
-  static constexpr uint32_t p = v + Cfg<S>::kVSlots * kSlotBytes;
+  static constexpr uint32_t qk = q + Width<R>::kQBytes;
+  static constexpr uint32_t v = qk + Cfg<S, R>::kQkSlots * kSlotBytes;
+  static constexpr uint32_t p = v + Cfg<S, R>::kVSlots * kSlotBytes;
   // float [2][S][128] row max (double-buffered by group parity) + [S][128] l
-  static constexpr uint32_t xch = p + Cfg<S>::kPRegion;
+  static constexpr uint32_t xch = p + Cfg<S, R>::kPRegion;
   static constexpr uint32_t bars = xch + 3 * S * 128 * 4;
   static constexpr uint32_t nbars = 48;
   static constexpr uint32_t misc = bars + nbars * 8;  // tmem slot, abort flag
-  static_assert(Cfg<S>::kQkSlots <= 6 && Cfg<S>::kVSlots <= 6, "barrier arrays hold 6 slots");
+  static_assert(Cfg<S, R>::kQkSlots <= 6 && Cfg<S, R>::kVSlots <= 6, "barrier arrays hold 6 slots");
   static constexpr uint32_t total = misc + 64;
   static constexpr uint32_t alloc = total + 1024;     // alignment slack
 };
@@ -216,13 +228,16 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk16) {
   return row * 128 + ((chunk16 ^ (row & 7)) << 4);
 }
 
-template <int S>
+template <int S, int R>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_q, RunParams p) {
   using namespace ptx;
-  using L = Smem<S>;
-  using C = Cfg<S>;
+  using L = Smem<S, R>;
+  using C = Cfg<S, R>;
+  using Wd = Width<R>;
+  static_assert(S == 1 || R == 512, "two shards in one launch split r = 512");
+  constexpr int kChunks = Wd::kChunks;
   extern __shared__ uint8_t smem_raw[];
   MLA_TRACE_CTA(0);
 
@@ -352,7 +367,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int rows[kGroupPages];
         for (int q = 0; q < kGroupPages; ++q) rows[q] = page_row(g.b, g.page + q, q < g.npages);
         for (int q = 0; q < kGroupPages && ok; ++q) {
-          for (int nb = 0; nb < 2 && ok; ++nb, ++vc) {
+          for (int nb = 0; nb < Wd::kNBlocks && ok; ++nb, ++vc) {
             const int slot = vc % C::kVSlots;
             if (vc >= (uint32_t)C::kVSlots)
               ok = mbar_wait(bar(B_V_FREE + slot), ((vc / C::kVSlots) - 1) & 1, p.wait_limit_ns);
@@ -438,7 +453,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = mbar_wait(bar(B_P_FULL_HI), gi & 1, p.wait_limit_ns);  // pages 2, 3 in the shared P buffer
             if (!ok) break;
           }
-          for (int nb = 0; nb < 2 && ok; ++nb, ++vc) {
+          for (int nb = 0; nb < Wd::kNBlocks && ok; ++nb, ++vc) {
             const int shard = S == 2 ? nb : 0;
             const int slot = vc % C::kVSlots;
             ok = mbar_wait(bar(B_V_FULL + slot), (vc / C::kVSlots) & 1, p.wait_limit_ns);
@@ -608,7 +623,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // O is rescaled (after the previous group's PV) before this group's
           // PV adds to it; both halves signal that through B_P_FULL.
           if (!g.first && __any_sync(0xffffffffu, rescale)) wait(B_PV_DONE, (gi - 1) & 1);
-          if (ok && !g.first && __any_sync(0xffffffffu, rescale)) rescale_o(0, 256);
+          if (ok && !g.first && __any_sync(0xffffffffu, rescale)) rescale_o(0, Wd::kOCols);
           if (half == 0) {
             // pages 0, 1: the previous group's PV must be done with pages 2, 3
             if (gi >= 1) wait(B_P_FREE_HI, (gi - 1) & 1);
@@ -678,7 +693,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int j = lane & 7;
           __half* oh = reinterpret_cast<__half*>(p.o_part);
 #pragma unroll 1
-          for (int c = 0; c < 256; c += 64) {
+          for (int c = 0; c < (int)Wd::kOCols; c += 64) {
             uint32_t o[64];
             tmem_ld32(tbase + lane_off + kTmemO + c, *reinterpret_cast<uint32_t(*)[32]>(o));
             tmem_ld32(tbase + lane_off + kTmemO + c + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
@@ -748,12 +763,13 @@ inline EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 row-major [rows, 576] with a (64 columns x 64 rows) 128B-swizzled box.
-inline bool make_rows_map(CUtensorMap* m, const void* ptr, uint64_t rows) {
+// 2-D bf16 row-major [rows, width] (width = r + d_rope) with a (64 columns x
+// 64 rows) 128B-swizzled box.
+inline bool make_rows_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t width = kWidth) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kWidth, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kWidth * 2};
+  cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)width * 2};
   cuuint32_t box[2] = {64, 64};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
@@ -763,23 +779,27 @@ inline bool make_rows_map(CUtensorMap* m, const void* ptr, uint64_t rows) {
 
 }  // namespace tc
 
+namespace tc {
+template <int S, int R>
+inline cudaError_t launch_decode_variant(const RunParams& p, const CUtensorMap& tm_kv, const CUtensorMap& tm_q,
+                                         cudaStream_t stream) {
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_tc_kernel<S, R>), (int)Smem<S, R>::alloc);
+  if (e != cudaSuccess) return e;
+  return launch_dependent(decode_tc_kernel<S, R>, dim3(2 * p.W), dim3(kThreads), Smem<S, R>::alloc, stream,
+                          tm_kv, tm_q, p);
+}
+}  // namespace tc
+
+// r = 512 with one or two latent shards, or r = 256 with one (a TPLA shard per GPU)
 inline cudaError_t launch_tc_decode(const RunParams& p, cudaStream_t stream) {
+  const uint64_t width = (uint64_t)p.r + p.dr;
   CUtensorMap tm_kv, tm_q;
-  if (!tc::make_rows_map(&tm_kv, p.kv, (uint64_t)p.num_blocks * 64)) return cudaErrorInvalidValue;
-  if (!tc::make_rows_map(&tm_q, p.q, (uint64_t)p.B * p.rows)) return cudaErrorInvalidValue;
-  cudaError_t e;
-  if (p.S == 1) {
-    e = ensure_smem_limit(reinterpret_cast<const void*>(tc::decode_tc_kernel<1>), (int)tc::Smem<1>::alloc);
-    if (e != cudaSuccess) return e;
-    e = launch_dependent(tc::decode_tc_kernel<1>, dim3(2 * p.W), dim3(tc::kThreads), tc::Smem<1>::alloc,
-                         stream, tm_kv, tm_q, p);
-  } else {
-    e = ensure_smem_limit(reinterpret_cast<const void*>(tc::decode_tc_kernel<2>), (int)tc::Smem<2>::alloc);
-    if (e != cudaSuccess) return e;
-    e = launch_dependent(tc::decode_tc_kernel<2>, dim3(2 * p.W), dim3(tc::kThreads), tc::Smem<2>::alloc,
-                         stream, tm_kv, tm_q, p);
-  }
-  return e;
+  if (!tc::make_rows_map(&tm_kv, p.kv, (uint64_t)p.num_blocks * 64, width)) return cudaErrorInvalidValue;
+  if (!tc::make_rows_map(&tm_q, p.q, (uint64_t)p.B * p.rows, width)) return cudaErrorInvalidValue;
+  if (p.r == 256 && p.S == 1) return tc::launch_decode_variant<1, 256>(p, tm_kv, tm_q, stream);
+  if (p.r != 512) return cudaErrorInvalidValue;
+  return p.S == 1 ? tc::launch_decode_variant<1, 512>(p, tm_kv, tm_q, stream)
+                  : tc::launch_decode_variant<2, 512>(p, tm_kv, tm_q, stream);
 }
 
 }  // namespace mla

@@ -1,4 +1,5 @@
-// tcgen05 per-head GEMMs of the bf16 decode path (r = 512, d_nope = d_v = 128):
+// tcgen05 per-head GEMMs of the bf16 decode path (r = 512 or 256, d_nope =
+// d_v = 128):
 //
 //   absorb : q_lat[row, :] = q_nope[row, h, :] . W_UK[h]            (K = 128, 512 outputs)
 //            (TransMLA abstract: W_UK is absorbed into the query)
@@ -46,7 +47,7 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk16) {
 }
 
 // ---------------------------------------------------------------------------
-// absorb: grid (H, 4 latent tiles, ceil(rows / 128)); block 256. One CTA per
+// absorb: grid (H, r / 128 latent tiles, ceil(rows / 128)); block 256. One CTA per
 // (head, 128-column latent tile): W_UK[h][:, tile] (32 KB, two MN-major groups
 // of 64 latent columns) as the A operand, q_nope rows [N][128] as 2 K-major
 // chunks; 8 MMAs into one tensor-memory accumulator. Small CTAs (~66 KB of
@@ -228,11 +229,11 @@ __global__ void __launch_bounds__(kCombineThreads, 1)
     fence_mbarrier_init_cluster();
     // the weights do not depend on the previous kernels: fetch them at once
     prefetch_tmap(&tm_wuv);
-    mbar_arrive_expect_tx_local(bar_w, 131072u);
+    mbar_arrive_expect_tx_local(bar_w, (uint32_t)p.r * 256u);  // r latent rows x 128 outputs, bf16
   }
   __syncwarp();
-  if (warp == 0 && lane < 4) {  // one 32 KB box per lane
-    const int j = lane >> 1, k = lane & 1;  // output columns [64 j, +64), latent rows [256 k, +256)
+  if (warp == 0 && lane < 2 * (p.r / 256)) {  // one 32 KB box per lane
+    const int j = lane & 1, k = lane >> 1;  // output columns [64 j, +64), latent rows [256 k, +256)
     tma_load_2d(base + CombineSmem::w + 65536 * j + 32768 * k, &tm_wuv, 64 * j, h * p.r + 256 * k, bar_w);
   }
   if (warp == 0) {
@@ -255,8 +256,9 @@ __global__ void __launch_bounds__(kCombineThreads, 1)
     const int64_t lstride = (int64_t)p.rows * S;
     const int64_t ostride = (int64_t)p.rows * p.r;
     const __half* opart = reinterpret_cast<const __half*>(p.o_part);
-    for (int it = threadIdx.x; it < n_pad * 16; it += kCombineThreads) {
-      const int i = it >> 4, slice = it & 15;
+    const int sl_shift = p.r == 512 ? 4 : 3;  // log2 of the 32-column items per row (r = 512 or 256)
+    for (int it = threadIdx.x; it < (n_pad << sl_shift); it += kCombineThreads) {
+      const int i = it >> sl_shift, slice = it & ((1 << sl_shift) - 1);
       const int c0 = 32 * slice;
       uint4 packed[4] = {};  // padding rows stay zero
       if (i < nrows) {
@@ -340,7 +342,7 @@ __global__ void __launch_bounds__(kCombineThreads, 1)
       const uint32_t idesc = idesc_bf16_f32(128, n_pad, 1, 0);
       const uint64_t a0 = smem_desc_sw128(base + CombineSmem::w, 65536, 1024);
       const uint64_t b0 = smem_desc_sw128(base + CombineSmem::x, 16, 1024);
-      for (int ks = 0; ks < 32; ++ks) {  // K = 512 = 32 x 16
+      for (int ks = 0; ks < p.r / 16; ++ks) {  // K = r in steps of 16
         const uint64_t ad = a0 + (uint64_t)(128 * ks);
         const uint64_t bd = b0 + (uint64_t)(((ks >> 2) * n_pad * 128) >> 4) + (uint64_t)(2 * (ks & 3));
         mma_f16<1>(tbase, ad, bd, idesc, ks > 0 ? 1u : 0u);
@@ -397,7 +399,7 @@ inline int pad16(int n) { return (n + 15) / 16 * 16; }
 
 }  // namespace hg
 
-// absorb on tensor cores (bf16, d_nope = 128, r = 512); also scans the lengths
+// absorb on tensor cores (bf16, d_nope = 128, r = 512 or 256); also scans the lengths
 inline cudaError_t launch_absorb_tc(const RunParams& p, cudaStream_t stream) {
   const int nbt = p.B * p.Lq;
   const int n_pad = hg::pad16(nbt < hg::kAbsorbMaxN ? nbt : hg::kAbsorbMaxN);
@@ -407,13 +409,13 @@ inline cudaError_t launch_absorb_tc(const RunParams& p, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(hg::absorb_tc_kernel), (int)hg::AbsorbSmem::alloc);
   if (e != cudaSuccess) return e;
-  const dim3 grid(p.H, 4, (nbt + hg::kAbsorbMaxN - 1) / hg::kAbsorbMaxN);  // r = 512: 4 latent tiles
+  const dim3 grid(p.H, p.r / 128, (nbt + hg::kAbsorbMaxN - 1) / hg::kAbsorbMaxN);  // 128-column latent tiles
   return launch_dependent(hg::absorb_tc_kernel, grid, dim3(hg::kThreads), hg::AbsorbSmem::alloc,
                               stream, tm_wuk, tm_qn, p, n_pad);
 }
 
 // split merge (bf16 o_lat into the query buffer) + up-projection on tensor
-// cores (bf16, r = 512, d_v = 128)
+// cores (bf16, r = 512 or 256, d_v = 128)
 inline cudaError_t launch_combine_tc(const RunParams& p, cudaStream_t stream) {
   const int nbt = p.B * p.Lq;
   const int rows_cta = hg::CombineSmem::kMaxRows;

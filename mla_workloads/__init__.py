@@ -57,7 +57,8 @@ from typing import Optional, Sequence
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "generate", "logical_cache", "pages_of", "stored_rows_fp8"]
+__all__ = ["Workload", "WORKLOADS", "generate", "logical_cache", "pages_of", "stored_rows_fp8",
+           "tpla_shard_columns", "tpla_shard_inputs"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -258,3 +259,23 @@ def logical_cache(inputs: dict, b: int, wl: Workload):
     ids = inputs["block_table"][b, :n].long()
     rows = inputs["kv_pool"][ids].reshape(n * P, wl.row_width)[:L]
     return rows[:, :wl.latent_rank], rows[:, wl.latent_rank:]
+
+
+def tpla_shard_columns(latent_rank: int, tp: int, g: int) -> slice:
+    """Latent columns of shard g of tp equal shards."""
+    w = latent_rank // tp
+    return slice(g * w, (g + 1) * w)
+
+
+def tpla_shard_inputs(inputs: dict, wl: Workload, tp: int, g: int) -> dict:
+    """The inputs one GPU of a tp-way TPLA group holds (layout only): the pool
+    rows with cKV narrowed to shard g's latent columns, followed by the full
+    RoPE key, [blocks, P, r / tp + dr]; W_UK[h][:, cols] and W_UV[h][cols, :];
+    queries, block table and lengths unchanged."""
+    cols = tpla_shard_columns(wl.latent_rank, tp, g)
+    pool = inputs["kv_pool"]
+    out = dict(inputs)
+    out["kv_pool"] = torch.cat([pool[..., cols], pool[..., wl.latent_rank:]], dim=-1).contiguous()
+    out["w_uk"] = inputs["w_uk"][:, :, cols].contiguous()
+    out["w_uv"] = inputs["w_uv"][:, cols, :].contiguous()
+    return out
