@@ -50,20 +50,21 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk16) {
 // absorb: grid (H, r / 128 latent tiles, ceil(rows / 128)); block 256. One CTA per
 // (head, 128-column latent tile): W_UK[h][:, tile] (32 KB, two MN-major groups
 // of 64 latent columns) as the A operand, q_nope rows [N][128] as 2 K-major
-// chunks; 8 MMAs into one tensor-memory accumulator. Small CTAs (~66 KB of
-// shared memory, 128 registers) so that several share an SM: 4 H CTAs spread
-// the 16.8 MB of W_UK over every SM instead of one 128 KB tile per SM.
+// chunks; 8 MMAs into one tensor-memory accumulator. Small CTAs (shared
+// memory sized to the query rows: ~41 KB for 32 rows, 64 registers) so that
+// four share an SM: the 4 H CTAs of a step (512 at 128 heads) run as one wave
+// and spread the 16.8 MB of W_UK over every SM.
 // ---------------------------------------------------------------------------
 constexpr int kAbsorbMaxN = 128;         // query rows per absorb CTA
 struct AbsorbSmem {
   static constexpr uint32_t w = 0;                             // 32 KB
-  static constexpr uint32_t x = 32768;                         // 2 x N x 128 B <= 32 KB
-  static constexpr uint32_t bars = x + 2 * kAbsorbMaxN * 128;
-  static constexpr uint32_t misc = bars + 64;
-  static constexpr uint32_t alloc = misc + 64 + 1024;
+  static constexpr uint32_t x = 32768;                         // 2 x n_pad x 128 B <= 32 KB
+  static constexpr uint32_t bars(int n_pad) { return x + 2u * (uint32_t)n_pad * 128u; }
+  static constexpr uint32_t misc(int n_pad) { return bars(n_pad) + 64; }
+  static constexpr uint32_t alloc(int n_pad) { return misc(n_pad) + 64 + 1024; }
 };
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 4)
     absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_wuk,
                      const __grid_constant__ CUtensorMap tm_qn, RunParams p, int n_pad) {
   using namespace ptx;
@@ -77,8 +78,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int row0 = blockIdx.z * kAbsorbMaxN;
   const int nrows = min(kAbsorbMaxN, nbt - row0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar_w = base + AbsorbSmem::bars, bar_x = bar_w + 8, bar_done = bar_w + 16;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(gbase + AbsorbSmem::misc);
+  const uint32_t bar_w = base + AbsorbSmem::bars(n_pad), bar_x = bar_w + 8, bar_done = bar_w + 16;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(gbase + AbsorbSmem::misc(n_pad));
   const uint32_t tcols = n_pad <= 32 ? 32 : n_pad <= 64 ? 64 : 128;
   if (threadIdx.x == 0) {
     mbar_init(bar_w, 1);
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0 && lane < 2)
     tma_load_2d(base + AbsorbSmem::w + 16384 * lane, &tm_wuk, 128 * mt + 64 * lane, h * p.dn, bar_w);
   if (warp == 0) {
-    tmem_alloc<1>(base + AbsorbSmem::misc, tcols);
+    tmem_alloc<1>(base + AbsorbSmem::misc(n_pad), tcols);
     tmem_relinquish<1>();
   }
   tc_fence_before();
@@ -407,10 +408,12 @@ inline cudaError_t launch_absorb_tc(const RunParams& p, cudaStream_t stream) {
   if (!hg::make_map(&tm_wuk, p.w_uk, (uint64_t)p.H * p.dn, (uint64_t)p.r, 128)) return cudaErrorInvalidValue;
   if (!hg::make_map(&tm_qn, p.q_nope, (uint64_t)nbt, (uint64_t)p.H * p.dn, (uint32_t)n_pad))
     return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(hg::absorb_tc_kernel), (int)hg::AbsorbSmem::alloc);
+  const uint32_t smem = hg::AbsorbSmem::alloc(n_pad);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(hg::absorb_tc_kernel),
+                                    (int)hg::AbsorbSmem::alloc(hg::kAbsorbMaxN));
   if (e != cudaSuccess) return e;
   const dim3 grid(p.H, p.r / 128, (nbt + hg::kAbsorbMaxN - 1) / hg::kAbsorbMaxN);  // 128-column latent tiles
-  return launch_dependent(hg::absorb_tc_kernel, grid, dim3(hg::kThreads), hg::AbsorbSmem::alloc,
+  return launch_dependent(hg::absorb_tc_kernel, grid, dim3(hg::kThreads), smem,
                               stream, tm_wuk, tm_qn, p, n_pad);
 }
 
