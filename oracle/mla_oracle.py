@@ -48,6 +48,7 @@ __all__ = [
     "softmax_attention",
     "mla_decode",
     "mla_decode_rows",
+    "mla_prefill",
 ]
 
 
@@ -123,4 +124,38 @@ def mla_decode(q_nope: np.ndarray, q_rope: np.ndarray, ckv_seqs: Sequence[np.nda
     for bi, b in enumerate(bs):
         out[bi] = mla_decode_rows(q_nope[b], q_rope[b], ckv_seqs[b], krope_seqs[b],
                                   w_uk, w_uv, scale, hs, latent_shards)
+    return out
+
+
+def mla_prefill(q_nope: np.ndarray, q_rope: np.ndarray, kv_rows: np.ndarray,
+                cu_seqlens: Sequence[int], w_uk: np.ndarray, w_uv: np.ndarray, scale: float,
+                pairs: Optional[Iterable] = None) -> np.ndarray:
+    """Causal prefill in the MLA (non-absorbed) form over concatenated prompts.
+
+    TPLA abstract: prefill keeps the MLA form. Every prompt token is a query
+    over the prompt's own tokens up to itself; per head the keys and values
+    are materialised from the latent rows exactly as in mla_decode.
+
+    q_nope [T, H, dn], q_rope [T, H, dr], kv_rows [T, r + dr] (cKV columns
+    [0, r), the RoPE key after them), cu_seqlens [B + 1] (sequence b owns rows
+    [cu[b], cu[b+1])), w_uk [H, dn, r], w_uv [H, r, dv]. pairs: (token row,
+    head) pairs to compute, all of them by default. Returns [len(pairs), dv].
+    """
+    T, H, _ = q_nope.shape
+    r = w_uk.shape[2]
+    cu = [int(x) for x in cu_seqlens]
+    if pairs is None:
+        pairs = [(t, h) for t in range(T) for h in range(H)]
+    pairs = list(pairs)
+    out = np.zeros((len(pairs), w_uv.shape[2]), dtype=np.float64)
+    groups = {}
+    for i, (t, h) in enumerate(pairs):
+        b = max(k for k in range(len(cu) - 1) if cu[k] <= t)
+        groups.setdefault((b, h), []).append((i, t))
+    for (b, h), items in groups.items():
+        rows = kv_rows[cu[b]:cu[b + 1]]
+        k, v = materialise_kv(rows[:, :r], rows[:, r:], w_uk[h], w_uv[h])
+        for i, t in items:
+            q = np.concatenate([q_nope[t, h], q_rope[t, h]])
+            out[i] = softmax_attention(q, k, v, scale, t - cu[b] + 1)
     return out

@@ -344,3 +344,39 @@ def test_fp8_logical_cache_scales_codes_and_rope():
     ckv, kr = logical_cache_fp8(codes, rope, scales)
     assert np.array_equal(ckv, [[0.25, -0.5, 0.0], [8.0, 4.0 * 2.0 ** -9, -4.0]])
     assert np.array_equal(kr, [[0.25, -0.75], [2.0, 8.0]])
+
+
+def test_prefill_matches_brute_force_and_is_causal():
+    """The prefill oracle against scalar loops (every token of two short
+    prompts, every head): query t of a prompt attends to the prompt's tokens
+    j <= t only, so each row is the brute-force decode of the prefix that ends
+    at t. Changing a later token must leave earlier rows unchanged."""
+    rng = np.random.default_rng(77)
+    H, r, dr, dn, dv = 2, 8, 2, 3, 4
+    lens = [5, 3]
+    T = sum(lens)
+    cu = [0, 5, 8]
+    q_nope = rng.standard_normal((T, H, dn))
+    q_rope = rng.standard_normal((T, H, dr))
+    kv_rows = rng.standard_normal((T, r + dr))
+    w_uk = rng.standard_normal((H, dn, r)) / math.sqrt(r)
+    w_uv = rng.standard_normal((H, r, dv)) / math.sqrt(r)
+    scale = 0.37
+    got = mo.mla_prefill(q_nope, q_rope, kv_rows, cu, w_uk, w_uv, scale)
+    i = 0
+    for t in range(T):
+        b = 0 if t < 5 else 1
+        n = t - cu[b] + 1
+        prefix = kv_rows[cu[b]:cu[b] + n]
+        ref = _brute(q_nope[None, t:t + 1], q_rope[None, t:t + 1], [prefix[:, :r]], [prefix[:, r:]],
+                     w_uk, w_uv, scale)[0, 0]
+        for h in range(H):
+            assert np.allclose(got[i], ref[h], rtol=1e-12, atol=1e-13)
+            i += 1
+    # causality: the last token of prompt 0 changes, earlier rows do not
+    kv2 = kv_rows.copy()
+    kv2[4] += 3.0
+    got2 = mo.mla_prefill(q_nope, q_rope, kv2, cu, w_uk, w_uv, scale)
+    assert np.array_equal(got2[:8], got[:8])       # tokens 0..3 of prompt 0, both heads
+    assert not np.allclose(got2[8:10], got[8:10])  # token 4 sees its own change
+    assert np.array_equal(got2[10:], got[10:])     # prompt 1 is independent
