@@ -410,10 +410,142 @@ def reference_arm(args, wl, world, rank):
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
+PREFILL_METRIC = "MLA-form prefill: TFLOP/s vs B200 bf16 tensor roofline"
+
+
+def prefill_work(wl, lens):
+    """FLOPs of one causal prefill: the up-projection (K_nope and V of every
+    token and head) and the attention (query t of a prompt sees t + 1 keys:
+    QK over d_nope + d_rope, PV over d_v); bytes it must move at least."""
+    H, r, dr, dn, dv = wl.heads, wl.latent_rank, wl.rope_dim, wl.nope_dim, wl.v_dim
+    T = int(sum(lens))
+    pairs = sum(int(L) * (int(L) + 1) // 2 for L in lens)
+    uproj = 2 * T * r * (dn + dv) * H
+    attn = 2 * pairs * H * (dn + dr + dv)
+    io = 2 * (T * H * (dn + dr + dv) + T * (r + dr) + H * r * (dn + dv))
+    return {"flops": uproj + attn, "uproj_flops": uproj, "attn_flops": attn, "bytes": io}
+
+
+def prefill_main(args, wl, world, rank, local):
+    """One step = one MLA-form prefill of the workload's prompts (the prefill
+    row of the method; the headline metric is the decode step)."""
+    import torch
+    import mla_latent_kv_21_b200 as M
+    from mla_workloads import generate_prefill
+    dist = init_dist(world)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    peaks, peaks_kind = load_peaks()
+    inputs = generate_prefill(wl)
+    lens = inputs["seq_lens"].tolist()
+    work = prefill_work(wl, lens)
+    dev = {k: v.to(device) for k, v in inputs.items()}
+    dims = M.dims_for(wl.heads, wl.latent_rank, wl.rope_dim, wl.nope_dim, wl.v_dim, 1, wl.softmax_scale,
+                      wl.dtype, 1, wl.page_size)
+    plan = M.PrefillPlan(dims, lens).allocate_workspace(device)
+    T = sum(lens)
+    out = torch.empty((T, wl.heads, wl.v_dim), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(d=dev, o=out, events=None):
+        plan.run(d["q_nope"], d["q_rope"], d["kv_rows"], d["cu_seqlens"], d["w_uk"], d["w_uv"], o,
+                 stream.cuda_stream, events)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    if plan.read_status() != 0:
+        raise SystemExit("device status after warm-up: " + M.mla_status_string(plan.read_status()))
+    K = args.steps
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    sampler.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    w0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    w_head = time.time()
+    drv = DriverEvents()
+    ev = [(drv.create(), drv.create()) for _ in range(K)]
+    for i in range(K):
+        step(events=ev[i])
+    torch.cuda.synchronize(device)
+    if dist:
+        dist.barrier()
+    sampler.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / K, dist, device)
+    attn_s = statistics.mean(drv.elapsed_ms(a, b) for a, b in ev) * 1e-3
+    drv.destroy()
+    if plan.read_status() != 0:
+        raise SystemExit("device status after timing")
+    # end to end with host buffers: the prompts' inputs in, the output back, every step
+    host = {k: inputs[k].pin_memory() for k in ("q_nope", "q_rope", "kv_rows", "cu_seqlens")}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    dset = {k: torch.empty_like(dev[k]) for k in host}
+    Ke = max(1, min(K, 10))
+    torch.cuda.synchronize(device)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(Ke):
+        for k, t in host.items():
+            dset[k].copy_(t, non_blocking=True)
+        step(d={**dev, **dset})
+        out_host.copy_(out, non_blocking=True)
+    x1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / Ke, dist, device)
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    value = world * work["flops"] / (ms * 1e-3) / 1e12
+    achieved = work["attn_flops"] / attn_s / 1e12
+    line = {
+        "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": len(lens), "prompt_tokens": lens, "heads": wl.heads,
+                   "latent_rank": wl.latent_rank, "rope_dim": wl.rope_dim, "nope_dim": wl.nope_dim,
+                   "v_dim": wl.v_dim, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"K_nope / V workspace {plan.workspace_bytes / 1e9:.2f} GB, larger than L2"},
+        "step_tflop": work["flops"] / 1e12,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "prefill attention",
+                     "peak_source": f"{peaks_kind} (bf16 sustained: a multi-ms kernel timed in a loop)",
+                     "attn_us": attn_s * 1e6, "attn_launches_timed": K},
+        "e2e": {"value": world * work["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "us_per_step": e2e_ms * 1e3,
+                "steps": Ke},
+        "gpu_launches": 2 * K,
+        "clocks": sampler.summary(w0, w_head),
+    }
+    emit(line, rank)
+    plan.close()
+    if dist:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_env()
-    from mla_workloads import WORKLOADS, generate
+    from mla_workloads import PREFILL_WORKLOADS, WORKLOADS, generate
+    if args.workload in PREFILL_WORKLOADS:
+        if args.impl == "reference":
+            emit({"impl": "reference", "unavailable": "the oracle arm times the decode step; prefill has no "
+                  "reference arm"}, rank)
+            return
+        pwl = PREFILL_WORKLOADS[args.workload]
+        if args.batch:
+            pwl = pwl.with_(batch=args.batch)
+        if args.context:
+            pwl = pwl.with_(context=args.context)
+        prefill_main(args, pwl, world, rank, local)
+        return
     wl = WORKLOADS[args.workload]
     if args.batch:
         wl = wl.with_(batch=args.batch)

@@ -260,6 +260,50 @@ mla_status_t mla_decode_selftest_timeout(mla_plan_t plan,
                                          void* out, void* workspace, size_t workspace_bytes,
                                          uint64_t wait_limit_ns, void* stream);
 
+/* ---- Prefill in the MLA (non-absorbed) form -------------------------------
+ * TPLA's abstract keeps the MLA form for the compute-bound prefill and the
+ * absorbed / TPLA form for the memory-bound decode. mla_prefill_run computes,
+ * for a batch of prompts, causal attention of every prompt token over the
+ * prompt's own tokens with per-head keys and values recovered from the latent
+ * rows:
+ *   K[h,t] = [cKV[t] . W_UK[h]^T || k_rope[t]],   V[h,t] = cKV[t] . W_UV[h]
+ *   out[t,h,:] = softmax_{j <= t}(scale q[t,h] . K[h,j]) . V[h, :]
+ * with q = [q_nope || q_rope] (TransMLA abstract: keys and values come from the
+ * latent by up-projection). The tokens of all prompts are concatenated:
+ * sequence b owns rows [cu[b], cu[b+1]) of
+ *   q_nope [T, H, d_nope], q_rope [T, H, d_rope], out [T, H, d_v] and
+ *   kv_rows [T, r + d_rope] (the prompt tokens' latent rows, the same rows the
+ *   caller writes into the paged cache; columns [0, r) cKV, [r, r + d_rope)
+ *   the RoPE key after RoPE).
+ * cu_seqlens_dev int32 [B + 1] (device) must hold the plan's lengths' prefix
+ * sums. The workspace (caller-owned) holds the up-projected K_nope and V,
+ * 2 T H (d_nope + d_v) bytes, plus a 1 KB header whose status word reports
+ * device-side errors (read it with mla_decode_read_status).
+ * Supported: bf16, r = 512, d_rope = 64, d_nope = d_v = 128, one latent shard
+ * (else MLA_ERR_UNSUPPORTED); dims.q_len and dims.page_size are not used. */
+typedef struct mla_prefill_plan* mla_prefill_plan_t;
+
+mla_status_t mla_prefill_plan(const mla_dims_t* dims, int32_t batch, const int32_t* seq_lens_host,
+                              mla_prefill_plan_t* plan_out, size_t* workspace_bytes);
+
+/* Enqueues the prefill on `stream` (two kernels: the up-projection, then the
+ * causal attention); all pointers but `plan` are device pointers. */
+mla_status_t mla_prefill_run(mla_prefill_plan_t plan, const void* q_nope, const void* q_rope,
+                             const void* kv_rows, const int32_t* cu_seqlens_dev,
+                             const void* w_uk, const void* w_uv, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* mla_prefill_run with options; opts may be NULL. The two events of
+ * mla_run_options_t are recorded around the attention kernel (the dominant
+ * kernel of a prefill). */
+mla_status_t mla_prefill_run_ex(mla_prefill_plan_t plan, const void* q_nope, const void* q_rope,
+                                const void* kv_rows, const int32_t* cu_seqlens_dev,
+                                const void* w_uk, const void* w_uv, void* out,
+                                void* workspace, size_t workspace_bytes, void* stream,
+                                const mla_run_options_t* opts);
+
+void mla_prefill_plan_destroy(mla_prefill_plan_t plan);
+
 /* Clears the workspace header (status word) with an async memset on `stream`.
  * Call once after allocating a workspace, before its first run. */
 mla_status_t mla_workspace_init(void* workspace, size_t workspace_bytes, void* stream);

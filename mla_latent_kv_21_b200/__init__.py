@@ -7,5 +7,5 @@ library and raises ImportError if it has not been built.
 
 from ._lib import *  # noqa: F401,F403
 from ._lib import MlaError, EXPORTED, LIB_PATH  # noqa: F401
-from .api import DecodePlan, dims_for  # noqa: F401
+from .api import DecodePlan, PrefillPlan, dims_for  # noqa: F401
 from .tpla import TplaShardPlan, shard_dims  # noqa: F401

@@ -45,7 +45,8 @@ EXPORTED = (
     "mla_decode_plan", "mla_decode_plan_ex", "mla_decode_run", "mla_decode_run_ex",
     "mla_decode_run_fp8", "mla_decode_run_no_alloc", "mla_decode_selftest_timeout", "mla_workspace_init",
     "mla_decode_read_status", "mla_plan_get_info", "mla_plan_segments", "mla_plan_destroy",
-    "mla_status_string", "mla_abi_version",
+    "mla_status_string", "mla_abi_version", "mla_prefill_plan", "mla_prefill_run",
+    "mla_prefill_run_ex", "mla_prefill_plan_destroy",
 )
 
 
@@ -102,6 +103,16 @@ _lib.mla_decode_run_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _v
 _lib.mla_decode_selftest_timeout.restype = ctypes.c_int
 _lib.mla_decode_selftest_timeout.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp,
                                              _vp, _sz, ctypes.c_uint64, _vp]
+_lib.mla_prefill_plan.restype = ctypes.c_int
+_lib.mla_prefill_plan.argtypes = [ctypes.POINTER(mla_dims_t), _i32, _i32p, ctypes.POINTER(_vp),
+                                  ctypes.POINTER(_sz)]
+_lib.mla_prefill_run.restype = ctypes.c_int
+_lib.mla_prefill_run.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.mla_prefill_run_ex.restype = ctypes.c_int
+_lib.mla_prefill_run_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
+                                    ctypes.POINTER(mla_run_options_t)]
+_lib.mla_prefill_plan_destroy.restype = None
+_lib.mla_prefill_plan_destroy.argtypes = [_vp]
 _lib.mla_workspace_init.restype = ctypes.c_int
 _lib.mla_workspace_init.argtypes = [_vp, _sz, _vp]
 _lib.mla_decode_read_status.restype = ctypes.c_int
@@ -212,6 +223,31 @@ def mla_decode_selftest_timeout(plan, q_nope, q_rope, kv_cache, num_blocks, bloc
                                             block_table_stride, seq_lens_dev, w_uk, w_uv, out,
                                             workspace, workspace_bytes, wait_limit_ns, stream),
            "mla_decode_selftest_timeout")
+
+
+def mla_prefill_plan(dims: mla_dims_t, seq_lens_host: Sequence[int]):
+    """-> (plan handle, workspace bytes) of a causal MLA-form prefill."""
+    plan = _vp()
+    ws = _sz()
+    arr = _lens_array(seq_lens_host)
+    _check(_lib.mla_prefill_plan(ctypes.byref(dims), len(seq_lens_host), arr, ctypes.byref(plan),
+                                 ctypes.byref(ws)), "mla_prefill_plan")
+    return plan.value, ws.value
+
+
+def mla_prefill_run(plan, q_nope, q_rope, kv_rows, cu_seqlens, w_uk, w_uv, out, workspace,
+                    workspace_bytes, stream=0, attn_start_event=None, attn_stop_event=None) -> None:
+    if attn_start_event is None and attn_stop_event is None:
+        _check(_lib.mla_prefill_run(plan, q_nope, q_rope, kv_rows, cu_seqlens, w_uk, w_uv, out, workspace,
+                                    workspace_bytes, stream), "mla_prefill_run")
+        return
+    opts = mla_run_options_t(attn_start_event, attn_stop_event)
+    _check(_lib.mla_prefill_run_ex(plan, q_nope, q_rope, kv_rows, cu_seqlens, w_uk, w_uv, out, workspace,
+                                   workspace_bytes, stream, ctypes.byref(opts)), "mla_prefill_run_ex")
+
+
+def mla_prefill_plan_destroy(plan) -> None:
+    _lib.mla_prefill_plan_destroy(plan)
 
 
 def mla_workspace_init(workspace, workspace_bytes, stream=0) -> None:

@@ -130,3 +130,64 @@ class DecodePlan:
             self.close()
         except Exception:
             pass
+
+
+class PrefillPlan:
+    """Owns one prefill plan handle and its device workspace tensor (the
+    up-projected per-head keys and values)."""
+
+    def __init__(self, dims: L.mla_dims_t, seq_lens_host: Sequence[int]):
+        self.dims = dims
+        self.lens = [int(x) for x in seq_lens_host]
+        self.handle, self.workspace_bytes = L.mla_prefill_plan(dims, self.lens)
+        self.workspace = None
+
+    def allocate_workspace(self, device) -> "PrefillPlan":
+        import torch
+        self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=device)
+        L.mla_workspace_init(self.workspace.data_ptr(), self.workspace_bytes,
+                             torch.cuda.current_stream(device).cuda_stream)
+        return self
+
+    def run(self, q_nope, q_rope, kv_rows, cu_seqlens, w_uk, w_uv, out, stream: Optional[int] = None,
+            attn_events=None) -> None:
+        """q_nope [T, H, dn], q_rope [T, H, dr], kv_rows [T, r + dr], cu_seqlens int32 [B + 1],
+        w_uk [H, dn, r], w_uv [H, r, dv], out [T, H, dv]: contiguous CUDA tensors."""
+        import torch
+        d, T = self.dims, sum(self.lens)
+        H, r, dr, dn, dv = d.num_heads, d.latent_rank, d.rope_dim, d.nope_dim, d.v_dim
+        bf = torch.bfloat16
+        for name, t, dtype, shape in (("q_nope", q_nope, bf, (T, H, dn)), ("q_rope", q_rope, bf, (T, H, dr)),
+                                      ("kv_rows", kv_rows, bf, (T, r + dr)),
+                                      ("cu_seqlens", cu_seqlens, torch.int32, (len(self.lens) + 1,)),
+                                      ("w_uk", w_uk, bf, (H, dn, r)), ("w_uv", w_uv, bf, (H, r, dv)),
+                                      ("out", out, bf, (T, H, dv))):
+            if t.dtype != dtype or tuple(t.shape) != shape:
+                raise ValueError(f"{name}: {t.dtype} {tuple(t.shape)}, the plan needs {dtype} {shape}")
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if self.workspace is None:
+            self.allocate_workspace(q_nope.device)
+        if stream is None:
+            stream = torch.cuda.current_stream(q_nope.device).cuda_stream
+        ev0, ev1 = (None, None) if attn_events is None else attn_events
+        L.mla_prefill_run(self.handle, q_nope.data_ptr(), q_rope.data_ptr(), kv_rows.data_ptr(),
+                          cu_seqlens.data_ptr(), w_uk.data_ptr(), w_uv.data_ptr(), out.data_ptr(),
+                          self.workspace.data_ptr(), self.workspace_bytes, stream, ev0, ev1)
+
+    def read_status(self, stream: Optional[int] = None) -> int:
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream(self.workspace.device).cuda_stream
+        return L.mla_decode_read_status(self.workspace.data_ptr(), stream)
+
+    def close(self) -> None:
+        if self.handle:
+            L.mla_prefill_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

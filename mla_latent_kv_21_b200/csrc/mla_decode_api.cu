@@ -13,6 +13,7 @@
 #include "tc_decode.cuh"
 #include "tc_decode_f8.cuh"
 #include "tc_head_gemm.cuh"
+#include "tc_prefill.cuh"
 
 using namespace mla;
 
@@ -352,6 +353,99 @@ mla_status_t mla_decode_selftest_timeout(mla_plan_t plan, const void* q_nope, co
                   block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace, workspace_bytes, stream_,
                   nullptr, k);
 }
+
+}  // extern "C"
+
+struct mla_prefill_plan {
+  mla_dims_t dims;
+  int32_t B;
+  int64_t T;
+  int32_t max_len;
+  size_t k_off, v_off, total;
+};
+
+extern "C" {
+
+mla_status_t mla_prefill_plan(const mla_dims_t* dims, int32_t batch, const int32_t* seq_lens_host,
+                              mla_prefill_plan_t* plan_out, size_t* workspace_bytes) {
+  if (!dims || !seq_lens_host || !plan_out || batch < 1) return MLA_ERR_INVALID_ARG;
+  *plan_out = nullptr;
+  const mla_dims_t& d = *dims;
+  if (d.num_heads < 1 || !std::isfinite(d.softmax_scale) || d.softmax_scale <= 0.f) return MLA_ERR_INVALID_ARG;
+  if (d.dtype != MLA_BF16 || d.latent_rank != 512 || d.rope_dim != 64 || d.nope_dim != 128 || d.v_dim != 128 ||
+      d.latent_shards != 1)
+    return MLA_ERR_UNSUPPORTED;
+  int64_t T = 0;
+  int32_t mx = 0;
+  for (int b = 0; b < batch; ++b) {
+    if (seq_lens_host[b] < 1) return MLA_ERR_INVALID_ARG;
+    T += seq_lens_host[b];
+    mx = std::max(mx, seq_lens_host[b]);
+  }
+  // row coordinates of the K_nope / V workspace ([H * T, 128]) are 32-bit
+  if ((int64_t)d.num_heads * (T + pf::kTile) >= (int64_t(1) << 31)) return MLA_ERR_UNSUPPORTED;
+  struct mla_prefill_plan* p = new (std::nothrow) struct mla_prefill_plan();
+  if (!p) return MLA_ERR_INVALID_ARG;
+  p->dims = d;
+  p->B = batch;
+  p->T = T;
+  p->max_len = mx;
+  p->k_off = 1024;
+  p->v_off = align_up(p->k_off + (size_t)T * d.num_heads * d.nope_dim * 2, 1024);
+  p->total = align_up(p->v_off + (size_t)T * d.num_heads * d.v_dim * 2, 1024);
+  *plan_out = p;
+  if (workspace_bytes) *workspace_bytes = p->total;
+  return MLA_OK;
+}
+
+mla_status_t mla_prefill_run(mla_prefill_plan_t plan, const void* q_nope, const void* q_rope,
+                             const void* kv_rows, const int32_t* cu_seqlens_dev, const void* w_uk,
+                             const void* w_uv, void* out, void* workspace, size_t workspace_bytes,
+                             void* stream_) {
+  return mla_prefill_run_ex(plan, q_nope, q_rope, kv_rows, cu_seqlens_dev, w_uk, w_uv, out, workspace,
+                            workspace_bytes, stream_, nullptr);
+}
+
+mla_status_t mla_prefill_run_ex(mla_prefill_plan_t plan, const void* q_nope, const void* q_rope,
+                                const void* kv_rows, const int32_t* cu_seqlens_dev, const void* w_uk,
+                                const void* w_uv, void* out, void* workspace, size_t workspace_bytes,
+                                void* stream_, const mla_run_options_t* opts) {
+  if (!plan || !q_nope || !q_rope || !kv_rows || !cu_seqlens_dev || !w_uk || !w_uv || !out || !workspace)
+    return MLA_ERR_INVALID_ARG;
+  if (workspace_bytes < plan->total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  const mla_dims_t& d = plan->dims;
+  char* ws = static_cast<char*>(workspace);
+  PrefillParams p{};
+  p.q_nope = q_nope;
+  p.q_rope = q_rope;
+  p.kv = kv_rows;
+  p.cu_seqlens = cu_seqlens_dev;
+  p.w_uk = w_uk;
+  p.w_uv = w_uv;
+  p.out = out;
+  p.status = reinterpret_cast<int32_t*>(ws);
+  p.k_nope = ws + plan->k_off;
+  p.v = ws + plan->v_off;
+  p.T = plan->T;
+  p.B = plan->B;
+  p.H = d.num_heads;
+  p.r = d.latent_rank;
+  p.dr = d.rope_dim;
+  p.dn = d.nope_dim;
+  p.dv = d.v_dim;
+  p.num_q_tiles = (plan->max_len + pf::kTile - 1) / pf::kTile;
+  p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  p.wait_limit_ns = ptx::kWaitLimitNs;
+  cudaEvent_t ev0 = opts ? static_cast<cudaEvent_t>(opts->decode_start_event) : nullptr;
+  cudaEvent_t ev1 = opts ? static_cast<cudaEvent_t>(opts->decode_stop_event) : nullptr;
+  if (launch_prefill(p, static_cast<cudaStream_t>(stream_), ev0, ev1) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
+void mla_prefill_plan_destroy(mla_prefill_plan_t plan) { delete plan; }
 
 mla_status_t mla_workspace_init(void* workspace, size_t workspace_bytes, void* stream_) {
   if (!workspace || workspace_bytes < 1024) return MLA_ERR_INVALID_ARG;

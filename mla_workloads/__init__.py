@@ -58,7 +58,7 @@ from typing import Optional, Sequence
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "generate", "logical_cache", "pages_of", "stored_rows_fp8",
-           "tpla_shard_columns", "tpla_shard_inputs"]
+           "tpla_shard_columns", "tpla_shard_inputs", "PREFILL_WORKLOADS", "generate_prefill"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -278,4 +278,38 @@ def tpla_shard_inputs(inputs: dict, wl: Workload, tp: int, g: int) -> dict:
     out["kv_pool"] = torch.cat([pool[..., cols], pool[..., wl.latent_rank:]], dim=-1).contiguous()
     out["w_uk"] = inputs["w_uk"][:, :, cols].contiguous()
     out["w_uv"] = inputs["w_uv"][:, cols, :].contiguous()
+    return out
+
+
+# Prefill workloads (MLA form; the prompt attends to itself causally): the
+# DeepSeek-V3 attention shape on prompts of 8K tokens.
+PREFILL_WORKLOADS = {
+    "deepseek_v3_prefill": Workload("deepseek_v3_prefill", seed=6, batch=2, q_len=1, heads=128,
+                                    latent_rank=512, rope_dim=64, nope_dim=128, v_dim=128,
+                                    context=8192),
+}
+_TAG_PQN, _TAG_PQR = 7, 8
+
+
+def generate_prefill(wl: Workload, seq_lens: Optional[Sequence[int]] = None) -> dict:
+    """Prefill inputs as CPU tensors: the prompts' tokens concatenated.
+
+    q_nope [T, H, dn], q_rope [T, H, dr] ~ N(0, 1); kv_rows [T, r + dr] (the
+    prompts' latent rows: per sequence the same N(0, 1) draw as a decode
+    workload's cache rows); W_UK, W_UV ~ N(0, 1/r); seq_lens int32 [B];
+    cu_seqlens int32 [B + 1] (prefix sums)."""
+    lens = draw_lengths(wl) if seq_lens is None else torch.as_tensor(list(seq_lens), dtype=torch.int32)
+    T = int(lens.sum())
+    dt = wl.torch_dtype
+    r, dr, dn, dv, H = wl.latent_rank, wl.rope_dim, wl.nope_dim, wl.v_dim, wl.heads
+    out = {"seq_lens": lens}
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(lens, 0)
+    out["cu_seqlens"] = cu
+    out["q_nope"] = torch.randn((T, H, dn), generator=_gen(wl.seed, _TAG_PQN)).to(dt)
+    out["q_rope"] = torch.randn((T, H, dr), generator=_gen(wl.seed, _TAG_PQR)).to(dt)
+    wstd = 1.0 / math.sqrt(r)
+    out["w_uk"] = (torch.randn((H, dn, r), generator=_gen(wl.seed, _TAG_WUK)) * wstd).to(dt)
+    out["w_uv"] = (torch.randn((H, r, dv), generator=_gen(wl.seed, _TAG_WUV)) * wstd).to(dt)
+    out["kv_rows"] = torch.cat([draw_sequence_rows(wl, b, int(L)) for b, L in enumerate(lens.tolist())], 0)
     return out

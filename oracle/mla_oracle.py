@@ -129,7 +129,7 @@ def mla_decode(q_nope: np.ndarray, q_rope: np.ndarray, ckv_seqs: Sequence[np.nda
 
 def mla_prefill(q_nope: np.ndarray, q_rope: np.ndarray, kv_rows: np.ndarray,
                 cu_seqlens: Sequence[int], w_uk: np.ndarray, w_uv: np.ndarray, scale: float,
-                pairs: Optional[Iterable] = None) -> np.ndarray:
+                pairs: Optional[Iterable] = None, abs_weighted: bool = False):
     """Causal prefill in the MLA (non-absorbed) form over concatenated prompts.
 
     TPLA abstract: prefill keeps the MLA form. Every prompt token is a query
@@ -139,7 +139,9 @@ def mla_prefill(q_nope: np.ndarray, q_rope: np.ndarray, kv_rows: np.ndarray,
     q_nope [T, H, dn], q_rope [T, H, dr], kv_rows [T, r + dr] (cKV columns
     [0, r), the RoPE key after them), cu_seqlens [B + 1] (sequence b owns rows
     [cu[b], cu[b+1])), w_uk [H, dn, r], w_uv [H, r, dv]. pairs: (token row,
-    head) pairs to compute, all of them by default. Returns [len(pairs), dv].
+    head) pairs to compute, all of them by default. Returns [len(pairs), dv];
+    with abs_weighted, also sum_j p_j |V_j| per row (the scale of any error
+    that rounds the values key by key), [len(pairs), dv].
     """
     T, H, _ = q_nope.shape
     r = w_uk.shape[2]
@@ -148,6 +150,7 @@ def mla_prefill(q_nope: np.ndarray, q_rope: np.ndarray, kv_rows: np.ndarray,
         pairs = [(t, h) for t in range(T) for h in range(H)]
     pairs = list(pairs)
     out = np.zeros((len(pairs), w_uv.shape[2]), dtype=np.float64)
+    aw = np.zeros_like(out)
     groups = {}
     for i, (t, h) in enumerate(pairs):
         b = max(k for k in range(len(cu) - 1) if cu[k] <= t)
@@ -157,5 +160,8 @@ def mla_prefill(q_nope: np.ndarray, q_rope: np.ndarray, kv_rows: np.ndarray,
         k, v = materialise_kv(rows[:, :r], rows[:, r:], w_uk[h], w_uv[h])
         for i, t in items:
             q = np.concatenate([q_nope[t, h], q_rope[t, h]])
-            out[i] = softmax_attention(q, k, v, scale, t - cu[b] + 1)
-    return out
+            n = t - cu[b] + 1
+            out[i] = softmax_attention(q, k, v, scale, n)
+            if abs_weighted:
+                aw[i] = softmax_attention(q, k, np.abs(v), scale, n)
+    return (out, aw) if abs_weighted else out

@@ -182,3 +182,30 @@ def assert_close(got, ref, dtype: str, what: str = ""):
         f"{what}: max_abs {max_abs:.3e} (tol {tol['max_abs']}), rel_fro {rel:.3e} "
         f"(tol {tol['rel_fro']:.3e}), element-wise bound ratio {ratio:.3f} (tol 1)")
     return max_abs, rel
+
+
+# Prefill (MLA form) has its own rounding steps: K_nope and V are materialised
+# in bf16 (the scores' and the values' roundings, key by key), P is bf16 and
+# the output bf16; q, k_rope and the latent rows are exact inputs. Rounding V
+# key by key moves an output element by at most u_bf16 sum_j p_j |V_j| (the
+# oracle's abs_weighted); the K_nope and P roundings are random terms of rms
+# RHO u_bf16 each relative to the row (as in the decode model). Element-wise
+# bound: u_bf16 |ref| + u_bf16 sum_j p_j |V_j| + ELEMENT_Z sigma rms(ref row),
+# sigma = hypot(RHO u, RHO u). Relative Frobenius and max-abs: the stated bf16
+# bounds.
+PREFILL_SIGMA = math.hypot(RHO * U["bf16"], RHO * U["bf16"])
+
+
+def assert_close_prefill(got, ref, abs_weighted, what: str = ""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    max_abs, rel = errors(got, ref)
+    rms_row = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
+    bound = U["bf16"] * (np.abs(ref) + np.asarray(abs_weighted)) + ELEMENT_Z * PREFILL_SIGMA * rms_row
+    ratio = float(np.max(np.abs(got - ref) / bound))
+    tol = TOL["bf16"]
+    assert rel <= tol["rel_fro"] and max_abs <= tol["max_abs"] and ratio <= 1.0, (
+        f"{what}: max_abs {max_abs:.3e} (tol {tol['max_abs']}), rel_fro {rel:.3e} (tol {tol['rel_fro']}), "
+        f"element-wise bound ratio {ratio:.3f} (tol 1)")
+    return max_abs, rel
