@@ -175,10 +175,12 @@ inline cudaError_t ensure_smem_limit(const void* func, int bytes) {
 
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel on the stream runs and waits for it in
-// grid_dependency_wait().
+// grid_dependency_wait(). pdl = false launches it in plain stream order (a
+// kernel bracketed by timing events: an event recorded between two kernels
+// chained this way does not mark the second one's start).
 template <typename... Params, typename... Args>
-inline cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
-                                    cudaStream_t stream, Args&&... args) {
+inline cudaError_t launch_dependent_opt(bool pdl, void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                                        cudaStream_t stream, Args&&... args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -186,10 +188,16 @@ inline cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 b
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... Params, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, Args&&... args) {
+  return launch_dependent_opt(true, kernel, grid, block, smem, stream, std::forward<Args>(args)...);
 }
 
 }  // namespace mla

@@ -277,10 +277,13 @@ mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, c
   cudaEvent_t ev_start = opts ? static_cast<cudaEvent_t>(opts->decode_start_event) : nullptr;
   cudaEvent_t ev_stop = opts ? static_cast<cudaEvent_t>(opts->decode_stop_event) : nullptr;
   if (ev_start && cudaEventRecord(ev_start, stream) != cudaSuccess) return MLA_ERR_CUDA;
+  // a decode bracketed by the caller's events runs in plain stream order, so
+  // that the start event marks its start
+  const bool pdl = ev_start == nullptr;
   if (p.fp8) {
-    if (launch_tc_decode_f8(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
+    if (launch_tc_decode_f8(p, stream, pdl) != cudaSuccess) return MLA_ERR_CUDA;
   } else if (plan->kernel == MLA_KERNEL_TCGEN05) {
-    if (launch_tc_decode(p, stream) != cudaSuccess) return MLA_ERR_CUDA;
+    if (launch_tc_decode(p, stream, pdl) != cudaSuccess) return MLA_ERR_CUDA;
   } else {
     const size_t smem = simt_decode_smem_bytes(p.r + p.dr, p.S, p.P);
     const dim3 gd(p.W, (p.rows + kSimtRowGroup - 1) / kSimtRowGroup);

@@ -782,24 +782,24 @@ inline bool make_rows_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64
 namespace tc {
 template <int S, int R>
 inline cudaError_t launch_decode_variant(const RunParams& p, const CUtensorMap& tm_kv, const CUtensorMap& tm_q,
-                                         cudaStream_t stream) {
+                                         cudaStream_t stream, bool pdl) {
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_tc_kernel<S, R>), (int)Smem<S, R>::alloc);
   if (e != cudaSuccess) return e;
-  return launch_dependent(decode_tc_kernel<S, R>, dim3(2 * p.W), dim3(kThreads), Smem<S, R>::alloc, stream,
-                          tm_kv, tm_q, p);
+  return launch_dependent_opt(pdl, decode_tc_kernel<S, R>, dim3(2 * p.W), dim3(kThreads), Smem<S, R>::alloc, stream,
+                              tm_kv, tm_q, p);
 }
 }  // namespace tc
 
 // r = 512 with one or two latent shards, or r = 256 with one (a TPLA shard per GPU)
-inline cudaError_t launch_tc_decode(const RunParams& p, cudaStream_t stream) {
+inline cudaError_t launch_tc_decode(const RunParams& p, cudaStream_t stream, bool pdl = true) {
   const uint64_t width = (uint64_t)p.r + p.dr;
   CUtensorMap tm_kv, tm_q;
   if (!tc::make_rows_map(&tm_kv, p.kv, (uint64_t)p.num_blocks * 64, width)) return cudaErrorInvalidValue;
   if (!tc::make_rows_map(&tm_q, p.q, (uint64_t)p.B * p.rows, width)) return cudaErrorInvalidValue;
-  if (p.r == 256 && p.S == 1) return tc::launch_decode_variant<1, 256>(p, tm_kv, tm_q, stream);
+  if (p.r == 256 && p.S == 1) return tc::launch_decode_variant<1, 256>(p, tm_kv, tm_q, stream, pdl);
   if (p.r != 512) return cudaErrorInvalidValue;
-  return p.S == 1 ? tc::launch_decode_variant<1, 512>(p, tm_kv, tm_q, stream)
-                  : tc::launch_decode_variant<2, 512>(p, tm_kv, tm_q, stream);
+  return p.S == 1 ? tc::launch_decode_variant<1, 512>(p, tm_kv, tm_q, stream, pdl)
+                  : tc::launch_decode_variant<2, 512>(p, tm_kv, tm_q, stream, pdl);
 }
 
 }  // namespace mla

@@ -720,7 +720,7 @@ inline bool make_map_bytes(CUtensorMap* m, const void* ptr, uint64_t rows, uint6
 
 }  // namespace tc8
 
-inline cudaError_t launch_tc_decode_f8(const RunParams& p, cudaStream_t stream) {
+inline cudaError_t launch_tc_decode_f8(const RunParams& p, cudaStream_t stream, bool pdl = true) {
   CUtensorMap tm_codes, tm_rope, tm_q;
   const uint64_t pool_rows = (uint64_t)p.num_blocks * 64;
   if (!tc8::make_map_bytes(&tm_codes, p.kv, pool_rows, 512, false)) return cudaErrorInvalidValue;
@@ -728,7 +728,7 @@ inline cudaError_t launch_tc_decode_f8(const RunParams& p, cudaStream_t stream) 
   if (!tc8::make_map_bytes(&tm_q, p.q, (uint64_t)p.B * p.rows, tc8::kQRowBytes, false)) return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(tc8::decode_f8_kernel), (int)tc8::Smem::alloc);
   if (e != cudaSuccess) return e;
-  return launch_dependent(tc8::decode_f8_kernel, dim3(2 * p.W), dim3(tc8::kThreads), tc8::Smem::alloc, stream,
+  return launch_dependent_opt(pdl, tc8::decode_f8_kernel, dim3(2 * p.W), dim3(tc8::kThreads), tc8::Smem::alloc, stream,
                           tm_codes, tm_rope, tm_q, p);
 }
 

@@ -563,8 +563,8 @@ inline cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream, c
   if (e != cudaSuccess) return e;
   if (ev_start && (e = cudaEventRecord(ev_start, stream)) != cudaSuccess) return e;
   const dim3 ga((unsigned)p.num_q_tiles, (unsigned)p.H, (unsigned)p.B);
-  e = launch_dependent(pf::attn_kernel, ga, dim3(pf::kThreads), pf::AttnSmem::alloc, stream, tm_qn, tm_qr, tm_kn,
-                       tm_kr, tm_v, p);
+  e = launch_dependent_opt(ev_start == nullptr, pf::attn_kernel, ga, dim3(pf::kThreads), pf::AttnSmem::alloc, stream,
+                           tm_qn, tm_qr, tm_kn, tm_kr, tm_v, p);
   if (e == cudaSuccess && ev_stop) e = cudaEventRecord(ev_stop, stream);
   return e;
 }
