@@ -49,6 +49,7 @@ __all__ = [
     "mla_decode",
     "mla_decode_rows",
     "mla_prefill",
+    "mla_decode_blasst",
 ]
 
 
@@ -165,3 +166,74 @@ def mla_prefill(q_nope: np.ndarray, q_rope: np.ndarray, kv_rows: np.ndarray,
             if abs_weighted:
                 aw[i] = softmax_attention(q, k, np.abs(v), scale, n)
     return (out, aw) if abs_weighted else out
+
+
+def mla_decode_blasst(q_nope_b: np.ndarray, q_rope_b: np.ndarray, ckv: np.ndarray,
+                      k_rope: np.ndarray, w_uk: np.ndarray, w_uv: np.ndarray, scale: float,
+                      segments: Sequence, skip_log2: float, group_keys: int = 256):
+    """Decode of one sequence (every head) with threshold skipping of key blocks.
+
+    BLASST abstract (kk6lht.com "GQA-to-MLA" listing): a fixed threshold and the
+    running maximum that the online softmax keeps identify negligible scores;
+    for them the exponentials, the value loads and the products with the values
+    are skipped. Read here for a blocked decode:
+
+    * the keys of the sequence are split into segments (``segments``: (first
+      key, end key) pairs, in key order, covering [0, L)), each processed with
+      its own running maxima; a segment's blocks are its consecutive runs of
+      ``group_keys`` keys from its first key (the last one shorter);
+    * for every query row (t, h), s_j = scale * q . K_h[j] over the keys it
+      may see (j <= L - Lq + t); its block maximum and running maximum are taken
+      in log2 units (s * log2 e);
+    * a row keeps a block when it sees a key there and either its running
+      maximum is still -inf or the block maximum is at least the running
+      maximum + skip_log2; a block is skipped when no row keeps it;
+    * every row's running maximum then takes the block maximum (a skipped
+      block's maxima are below it, so skipping leaves it unchanged);
+    * out = softmax over the row's visible keys in kept blocks, times V_h.
+
+    q_nope_b [Lq, H, dn], q_rope_b [Lq, H, dr], ckv [L, r], k_rope [L, dr],
+    w_uk [H, dn, r], w_uv [H, r, dv]. Returns (out [Lq, H, dv], kept [blocks],
+    margin [blocks]) with margin = the largest row value of block max - running
+    max - skip_log2 (the decision's distance from the threshold; +inf where a row
+    with no running maximum yet keeps the block).
+    """
+    Lq, H, _ = q_nope_b.shape
+    L = ckv.shape[0]
+    dv = w_uv.shape[2]
+    log2e = 1.0 / np.log(2.0)
+    scores = np.full((Lq, H, L), -np.inf)
+    values = []
+    for h in range(H):
+        k, v = materialise_kv(ckv, k_rope, w_uk[h], w_uv[h])
+        values.append(v)
+        for t in range(Lq):
+            n = L - Lq + t + 1
+            q = np.concatenate([q_nope_b[t, h], q_rope_b[t, h]])
+            scores[t, h, :n] = scale * (k[:n] @ q)
+    s2 = scores * log2e
+    included = np.zeros(L, dtype=bool)
+    kept, margins = [], []
+    for k0, k1 in segments:
+        runmax = np.full((Lq, H), -np.inf)
+        for g0 in range(k0, k1, group_keys):
+            g1 = min(g0 + group_keys, k1)
+            bm = s2[:, :, g0:g1].max(axis=2)
+            seen = np.isfinite(bm)
+            first = seen & np.isneginf(runmax)
+            cmp = np.where(seen & ~first, bm - runmax - skip_log2, -np.inf)
+            keep = bool(first.any() or (cmp >= 0).any())
+            kept.append(keep)
+            margins.append(np.inf if first.any() else float(cmp.max()))
+            runmax = np.maximum(runmax, bm)
+            if keep:
+                included[g0:g1] = True
+    out = np.zeros((Lq, H, dv))
+    for t in range(Lq):
+        n = L - Lq + t + 1
+        mask = included[:n]
+        for h in range(H):
+            s = scores[t, h, :n][mask]
+            p = np.exp(s - s.max())
+            out[t, h] = (p / p.sum()) @ values[h][:n][mask]
+    return out, np.array(kept), np.array(margins)

@@ -85,36 +85,7 @@ def test_run_rejects_null_and_small_workspace():
         L.mla_plan_destroy(plan)
 
 
-SEGMENT_COST_PAGES = 4  # places a sequence boundary takes on the partition's cost line
-
-
-def _reference_segments(lens, P, W):
-    """Independent recomputation of the split partition: lay the pages out on a
-    cost line where each sequence boundary takes SEGMENT_COST_PAGES places, cut
-    the line into W equal parts (floor), and start each worker at the first
-    real page at or after its cut (brute force over the pages)."""
-    pages = [-(-x // P) for x in lens]
-    bounds = [0]
-    for n in pages:
-        bounds.append(bounds[-1] + n)
-    G = bounds[-1]
-    pos = []  # cost-line position of every real page
-    for b, n in enumerate(pages):
-        pos.extend(bounds[b] + i + SEGMENT_COST_PAGES * b for i in range(n))
-    line = G + SEGMENT_COST_PAGES * (len(pages) - 1)
-
-    def start(w):
-        cut = w * line // W
-        return next((x for x, v in enumerate(pos) if v >= cut), G)
-
-    segs = []
-    for w in range(W):
-        a, e = start(w), start(w + 1)
-        for b in range(len(lens)):
-            lo, hi = max(a, bounds[b]), min(e, bounds[b + 1])
-            if lo < hi:
-                segs.append((w, b, lo - bounds[b], hi - bounds[b], w + b))
-    return segs, pages
+from harness_partition import reference_segments as _reference_segments  # noqa: E402
 
 
 @pytest.mark.parametrize("seed", range(12))

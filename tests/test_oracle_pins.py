@@ -380,3 +380,61 @@ def test_prefill_matches_brute_force_and_is_causal():
     assert np.array_equal(got2[:8], got[:8])       # tokens 0..3 of prompt 0, both heads
     assert not np.allclose(got2[8:10], got[8:10])  # token 4 sees its own change
     assert np.array_equal(got2[10:], got[10:])     # prompt 1 is independent
+
+
+def _blasst_problem(rng, L=12, Lq=1, H=2, r=8, dr=2, dn=3, dv=4):
+    q_nope = rng.standard_normal((Lq, H, dn))
+    q_rope = np.zeros((Lq, H, dr))
+    q_rope[:, :, 0] = 10.0
+    ckv = rng.standard_normal((L, r))
+    kr = np.zeros((L, dr))
+    kr[:, 0] = 1.0
+    w_uk = rng.standard_normal((H, dn, r)) / math.sqrt(r) * 0.1
+    w_uv = rng.standard_normal((H, r, dv)) / math.sqrt(r)
+    return q_nope, q_rope, ckv, kr, w_uk, w_uv
+
+
+def test_blasst_without_threshold_is_the_dense_decode():
+    rng = np.random.default_rng(90)
+    prob = _rand_problem(rng, B=1, Lq=2, lens=(23,))
+    q_nope, q_rope, ckv, kr, w_uk, w_uv = prob
+    dense = mo.mla_decode(q_nope, q_rope, ckv, kr, w_uk, w_uv, 0.4)[0]
+    for segs in ([(0, 23)], [(0, 9), (9, 23)]):
+        got, kept, _ = mo.mla_decode_blasst(q_nope[0], q_rope[0], ckv[0], kr[0], w_uk, w_uv, 0.4, segs,
+                                            -np.inf, group_keys=4)
+        assert kept.all()
+        assert np.allclose(got, dense, rtol=1e-12, atol=1e-14)
+
+
+def test_blasst_skips_exactly_the_negligible_block():
+    """Keys 4..7 score ~60 log2 units below the others for every row: with a
+    threshold of -10 that block (and only it) is skipped, and the output is the
+    brute-force attention over the kept keys. With the block's keys moved into
+    a segment of their own it is that segment's first block and is kept."""
+    rng = np.random.default_rng(91)
+    q_nope, q_rope, ckv, kr, w_uk, w_uv = _blasst_problem(rng)
+    kr[4:8, 0] = -5.0
+    scale = 0.5
+    got, kept, margin = mo.mla_decode_blasst(q_nope, q_rope, ckv, kr, w_uk, w_uv, scale, [(0, 12)],
+                                             -10.0, group_keys=4)
+    assert kept.tolist() == [True, False, True]
+    assert margin[1] < -20 and margin[2] > 5
+    keep = np.r_[0:4, 8:12]
+    ref = _brute(q_nope[None], q_rope[None], [ckv[keep]], [kr[keep]], w_uk, w_uv, scale)[0]
+    assert np.allclose(got, ref, rtol=1e-11, atol=1e-13)
+    # a segment that starts at key 4 keeps its first block
+    _, kept2, _ = mo.mla_decode_blasst(q_nope, q_rope, ckv, kr, w_uk, w_uv, scale, [(0, 4), (4, 12)],
+                                       -10.0, group_keys=4)
+    assert kept2.tolist() == [True, True, True]
+
+
+def test_blasst_keeps_a_block_that_one_row_needs():
+    """Only head 1 scores high on keys 4..7 (head 0 scores them very low): the
+    block is kept for both heads (the decision covers every row)."""
+    rng = np.random.default_rng(92)
+    q_nope, q_rope, ckv, kr, w_uk, w_uv = _blasst_problem(rng)
+    q_rope[0, 1, 1] = 10.0       # head 1 also reads the second RoPE column
+    kr[4:8, 0] = -5.0
+    kr[4:8, 1] = 8.0             # ... where keys 4..7 score high
+    _, kept, _ = mo.mla_decode_blasst(q_nope, q_rope, ckv, kr, w_uk, w_uv, 0.5, [(0, 12)], -10.0, group_keys=4)
+    assert kept.tolist() == [True, True, True]
