@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="oracle work for the cpu_baseline sample")
+    ap.add_argument("--blasst", type=float, default=None, metavar="LOG2",
+                    help="decode with threshold skipping of key groups below the running max + LOG2 (<= 0)")
     ap.add_argument("--tpla-shard", action="store_true",
                     help="TPLA workloads on one GPU: time one GPU's latent shard of the multi-GPU form "
                          "(no all-reduce: the other shards live on other GPUs)")
@@ -598,6 +600,9 @@ def main():
         if wl.dtype == "fp8":
             plan.run_fp8(q_nope, q_rope, dev["kv_codes"], dev["kv_rope"], dev["kv_scale"], block_table,
                          seq_lens, dev["w_uk"], dev["w_uv"], o, stream.cuda_stream, events)
+        elif args.blasst is not None:
+            plan.run_blasst(q_nope, q_rope, dev["kv_pool"], block_table, seq_lens, dev["w_uk"], dev["w_uv"], o,
+                            args.blasst, stream.cuda_stream, events)
         else:
             plan.run(q_nope, q_rope, dev["kv_pool"], block_table, seq_lens, dev["w_uk"], dev["w_uv"], o,
                      stream.cuda_stream, events)
@@ -767,6 +772,13 @@ def main():
         "gpu_launches": info.launches_per_run * K,
         "clocks": sampler.summary(w0, w_head),
     }
+    if args.blasst is not None:
+        # skip counters of the last step (every step of a plan makes the same decisions)
+        skipped, groups = plan.skip_counts()
+        line["blasst"] = {"skip_log2": args.blasst, "skipped_groups": skipped, "groups": groups,
+                          "sparsity": skipped / max(1, groups),
+                          "note": "threshold skipping: the result is the attention over the kept key groups"}
+        line["config"]["kernel"] += "+threshold_skipping"
 
     if rank == 0 and world == 1 and tp == 1 and not args.no_cpu_baseline:
         # the oracle as it stands on the host cores, bounded sample; its sampled

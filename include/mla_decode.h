@@ -240,6 +240,35 @@ mla_status_t mla_decode_run_no_alloc(mla_plan_t plan,
                                      const void* w_uk, const void* w_uv,
                                      void* out, void* stream);
 
+/* One decode step with threshold skipping of negligible key groups. The BLASST
+ * abstract (on the kk6lht.com "GQA-to-MLA" search listing) compares a fixed
+ * threshold with the running maximum the online softmax already keeps and
+ * skips, for blocks of scores found negligible, their exponentials, the value
+ * loads and the P.V products. Here the block is a group of 256 keys (4 pages)
+ * of one split segment, for all H * Lq query rows of the sequence together:
+ * the group is skipped when, for every row, its largest score in log2 units
+ * (score * softmax_scale * log2 e, over the keys the row may see) is below
+ * the row's running maximum over the segment's earlier groups plus skip_log2
+ * (a finite threshold <= 0, or -inf to skip nothing). A row's first group with
+ * a visible key in a segment is always kept. Groups start at each segment's
+ * first page, so which groups exist depends on the plan's split partition
+ * (mla_plan_segments); a plan gives the same result every run. The result is
+ * the attention over the kept keys (an approximation of the full step by
+ * design), merged across segments as in mla_decode_run. Plans: bf16 on the
+ * tensor-core kernel, r = 512, one latent shard (else MLA_ERR_UNSUPPORTED).
+ * The call also writes two int32 counters into the workspace header: the
+ * number of skipped groups (byte offset 8) and of all groups (offset 12).
+ * opts (may be NULL): timing events around the decode kernel, as for
+ * mla_decode_run_ex. */
+mla_status_t mla_decode_run_blasst(mla_plan_t plan,
+                                   const void* q_nope, const void* q_rope,
+                                   const void* kv_cache, int64_t num_blocks,
+                                   const int32_t* block_table, int32_t block_table_stride,
+                                   const int32_t* seq_lens_dev,
+                                   const void* w_uk, const void* w_uv,
+                                   void* out, void* workspace, size_t workspace_bytes,
+                                   float skip_log2, void* stream, const mla_run_options_t* opts);
+
 /* Self-test of the device-side timeout path (diagnostics; not a decode).
  * Runs one step of mla_decode_run on the same arguments, except that in the
  * split-KV decode kernel every bounded wait gives up after wait_limit_ns

@@ -43,7 +43,8 @@ MLA_KERNEL_TCGEN05 = 2
 # symbols declared in include/mla_decode.h
 EXPORTED = (
     "mla_decode_plan", "mla_decode_plan_ex", "mla_decode_run", "mla_decode_run_ex",
-    "mla_decode_run_fp8", "mla_decode_run_no_alloc", "mla_decode_selftest_timeout", "mla_workspace_init",
+    "mla_decode_run_fp8", "mla_decode_run_no_alloc", "mla_decode_selftest_timeout", "mla_decode_run_blasst",
+    "mla_workspace_init",
     "mla_decode_read_status", "mla_plan_get_info", "mla_plan_segments", "mla_plan_destroy",
     "mla_status_string", "mla_abi_version", "mla_prefill_plan", "mla_prefill_run",
     "mla_prefill_run_ex", "mla_prefill_plan_destroy",
@@ -100,6 +101,9 @@ _lib.mla_decode_run_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _i3
 _lib.mla_decode_run_no_alloc.restype = ctypes.c_int
 _lib.mla_decode_run_no_alloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp,
                                          _vp]
+_lib.mla_decode_run_blasst.restype = ctypes.c_int
+_lib.mla_decode_run_blasst.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz,
+                                       ctypes.c_float, _vp, ctypes.POINTER(mla_run_options_t)]
 _lib.mla_decode_selftest_timeout.restype = ctypes.c_int
 _lib.mla_decode_selftest_timeout.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp,
                                              _vp, _sz, ctypes.c_uint64, _vp]
@@ -212,6 +216,18 @@ def mla_decode_run_no_alloc(plan, q_nope, q_rope, kv_cache, num_blocks, block_ta
     _check(_lib.mla_decode_run_no_alloc(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,
                                         block_table_stride, seq_lens_dev, w_uk, w_uv, out,
                                         stream), "mla_decode_run_no_alloc")
+
+
+def mla_decode_run_blasst(plan, q_nope, q_rope, kv_cache, num_blocks, block_table, block_table_stride,
+                          seq_lens_dev, w_uk, w_uv, out, workspace, workspace_bytes, skip_log2,
+                          stream=0, decode_start_event=None, decode_stop_event=None) -> None:
+    """One decode step skipping key groups whose scores fall below the running
+    max + skip_log2 (log2 units) for every query row (see the C header)."""
+    opts = mla_run_options_t(decode_start_event, decode_stop_event)
+    _check(_lib.mla_decode_run_blasst(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,
+                                      block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace,
+                                      workspace_bytes, float(skip_log2), stream, ctypes.byref(opts)),
+           "mla_decode_run_blasst")
 
 
 def mla_decode_selftest_timeout(plan, q_nope, q_rope, kv_cache, num_blocks, block_table,

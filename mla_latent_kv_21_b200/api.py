@@ -114,6 +114,38 @@ class DecodePlan:
                              w_uk.data_ptr(), w_uv.data_ptr(), out.data_ptr(),
                              self.workspace.data_ptr(), self.workspace_bytes, stream, ev0, ev1)
 
+    def run_blasst(self, q_nope, q_rope, kv_pool, block_table, seq_lens, w_uk, w_uv, out, skip_log2: float,
+                   stream: Optional[int] = None, decode_events=None) -> None:
+        """A decode step with threshold skipping (mla_decode_run_blasst); the
+        arguments are those of run plus the threshold in log2 units (<= 0)."""
+        import torch
+        d = self.dims
+        act = torch.bfloat16
+        self._check_common(act, q_nope, q_rope, block_table, seq_lens, w_uk, w_uv, out)
+        self._check("kv_pool", kv_pool, act, (None, d.page_size, d.latent_rank + d.rope_dim))
+        for name, t in (("q_nope", q_nope), ("q_rope", q_rope), ("kv_pool", kv_pool),
+                        ("block_table", block_table), ("seq_lens", seq_lens), ("w_uk", w_uk),
+                        ("w_uv", w_uv), ("out", out)):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if self.workspace is None:
+            self.allocate_workspace(q_nope.device)
+        if stream is None:
+            stream = torch.cuda.current_stream(q_nope.device).cuda_stream
+        ev0, ev1 = (None, None) if decode_events is None else decode_events
+        L.mla_decode_run_blasst(self.handle, q_nope.data_ptr(), q_rope.data_ptr(), kv_pool.data_ptr(),
+                                kv_pool.shape[0], block_table.data_ptr(), block_table.shape[1],
+                                seq_lens.data_ptr(), w_uk.data_ptr(), w_uv.data_ptr(), out.data_ptr(),
+                                self.workspace.data_ptr(), self.workspace_bytes, skip_log2, stream, ev0, ev1)
+
+    def skip_counts(self):
+        """(skipped groups, groups) of the last threshold-skipping step (the
+        workspace header's counters; synchronises the device)."""
+        import torch
+        torch.cuda.synchronize(self.workspace.device)
+        c = self.workspace[8:16].view(torch.int32).cpu().tolist()
+        return c[0], c[1]
+
     def read_status(self, stream: Optional[int] = None) -> int:
         import torch
         if stream is None:

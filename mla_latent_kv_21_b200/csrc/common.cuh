@@ -133,6 +133,10 @@ struct RunParams {
   // self-test of the timeout path only: the decode kernel's softmax withholds
   // the release of its score buffers, so the QK issuer's wait runs out
   int32_t withhold_s_free;
+  // threshold skipping (the skipping decode only): log2 threshold below the
+  // running max, and the workspace counters (skipped groups, groups)
+  float skip_log2;
+  int32_t* skip_stats;
 };
 
 // True for a plan over the FP8 latent cache (host; defined with the ABI).

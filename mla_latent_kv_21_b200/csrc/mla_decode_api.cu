@@ -212,6 +212,8 @@ namespace {
 struct WaitKnobs {
   uint64_t limit_ns = ptx::kWaitLimitNs;
   int32_t withhold_s_free = 0;
+  bool skip = false;        // threshold-skipping decode
+  float skip_log2 = 0.f;
 };
 
 mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, const void* kv_cache,
@@ -261,6 +263,9 @@ mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, c
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
   p.wait_limit_ns = knobs.limit_ns;
   p.withhold_s_free = knobs.withhold_s_free;
+  p.skip_log2 = knobs.skip_log2;
+  p.skip_stats = reinterpret_cast<int32_t*>(ws + 8);
+  if (knobs.skip && cudaMemsetAsync(ws + 8, 0, 8, stream) != cudaSuccess) return MLA_ERR_CUDA;
 
   const bool bf16 = d.dtype == MLA_BF16;
   const int nbt = p.B * p.Lq;
@@ -283,7 +288,7 @@ mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, c
   if (p.fp8) {
     if (launch_tc_decode_f8(p, stream, pdl) != cudaSuccess) return MLA_ERR_CUDA;
   } else if (plan->kernel == MLA_KERNEL_TCGEN05) {
-    if (launch_tc_decode(p, stream, pdl) != cudaSuccess) return MLA_ERR_CUDA;
+    if (launch_tc_decode(p, stream, pdl, knobs.skip) != cudaSuccess) return MLA_ERR_CUDA;
   } else {
     const size_t smem = simt_decode_smem_bytes(p.r + p.dr, p.S, p.P);
     const dim3 gd(p.W, (p.rows + kSimtRowGroup - 1) / kSimtRowGroup);
@@ -338,6 +343,22 @@ mla_status_t mla_decode_run_fp8(mla_plan_t plan, const void* q_nope, const void*
   if (!plan || plan->dims.dtype != MLA_FP8_CACHE || !kv_rope || !kv_scale) return MLA_ERR_INVALID_ARG;
   return run_impl(plan, q_nope, q_rope, kv_codes, kv_rope, kv_scale, num_blocks, block_table,
                   block_table_stride, seq_lens_dev, w_uk, w_uv, out, workspace, workspace_bytes, stream_, opts);
+}
+
+mla_status_t mla_decode_run_blasst(mla_plan_t plan, const void* q_nope, const void* q_rope,
+                                   const void* kv_cache, int64_t num_blocks, const int32_t* block_table,
+                                   int32_t block_table_stride, const int32_t* seq_lens_dev, const void* w_uk,
+                                   const void* w_uv, void* out, void* workspace, size_t workspace_bytes,
+                                   float skip_log2, void* stream_, const mla_run_options_t* opts) {
+  if (!plan || plan->dims.dtype != MLA_BF16 || plan->kernel != MLA_KERNEL_TCGEN05 || plan->dims.latent_rank != 512 ||
+      plan->dims.latent_shards != 1)
+    return MLA_ERR_UNSUPPORTED;
+  if (!(skip_log2 <= 0.f)) return MLA_ERR_INVALID_ARG;  // NaN and positive thresholds refused
+  WaitKnobs k;
+  k.skip = true;
+  k.skip_log2 = skip_log2;
+  return run_impl(plan, q_nope, q_rope, kv_cache, nullptr, nullptr, num_blocks, block_table, block_table_stride,
+                  seq_lens_dev, w_uk, w_uv, out, workspace, workspace_bytes, stream_, opts, k);
 }
 
 mla_status_t mla_decode_selftest_timeout(mla_plan_t plan, const void* q_nope, const void* q_rope,

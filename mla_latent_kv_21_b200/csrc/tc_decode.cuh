@@ -108,7 +108,7 @@ struct Smem {
   // float [2][S][128] row max (double-buffered by group parity) + [S][128] l
   static constexpr uint32_t xch = p + Cfg<S, R>::kPRegion;
   static constexpr uint32_t bars = xch + 3 * S * 128 * 4;
-  static constexpr uint32_t nbars = 48;
+  static constexpr uint32_t nbars = 56;
   static constexpr uint32_t misc = bars + nbars * 8;  // tmem slot, abort flag
   static_assert(Cfg<S, R>::kQkSlots <= 6 && Cfg<S, R>::kVSlots <= 6, "barrier arrays hold 6 slots");
   static constexpr uint32_t total = misc + 64;
@@ -133,7 +133,10 @@ enum : int {
   B_P_FREE_HI = 35,   // both, count 1: PV is done with P of group pages 2, 3
   B_QC_FULL = 36,     // [9] leader, count 2 (+tx): query chunk k of the current segment
   B_P_FULL_HI = 45,   // leader, count 4 (shared P: pages 2, 3 written by 2 warps x 2 CTAs)
-  B_COUNT = 46
+  // threshold skipping (kSkip): the pair's keep / skip decision of group gi
+  B_DECIDE = 46,      // [2] both, count 1 (+4 tx bytes: the peer's vote), by group parity
+  B_VSEEN = 48,       // [2] both, count 1: the V producer has read the decision of group gi
+  B_COUNT = 50
 };
 
 // Optional event trace (compile with -DMLA_TRACE): SM clock of per-group events
@@ -228,7 +231,7 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk16) {
   return row * 128 + ((chunk16 ^ (row & 7)) << 4);
 }
 
-template <int S, int R>
+template <int S, int R, bool kSkip = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_q, RunParams p) {
@@ -237,6 +240,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   using C = Cfg<S, R>;
   using Wd = Width<R>;
   static_assert(S == 1 || R == 512, "two shards in one launch split r = 512");
+  static_assert(!kSkip || (S == 1 && C::kSharedP), "threshold skipping: one latent shard");
   constexpr int kChunks = Wd::kChunks;
   extern __shared__ uint8_t smem_raw[];
   MLA_TRACE_CTA(0);
@@ -263,6 +267,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::misc + 8);
+  // threshold skipping: votes [group parity][CTA rank] (nonzero: some row of
+  // that CTA keeps the group)
+  volatile uint32_t* votes = reinterpret_cast<volatile uint32_t*>(gbase + L::misc + 16);
+  auto pair_keeps = [&](int gi) { return (votes[2 * (gi & 1)] | votes[2 * (gi & 1) + 1]) != 0; };
   float* xch = reinterpret_cast<float*>(gbase + L::xch);
 
   if (threadIdx.x == 0) {
@@ -276,6 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     counts[B_P_FULL] = 8;
     counts[B_P_FULL_HI] = 4;
     counts[B_O_FREE] = 8;
+    counts[B_VSEEN] = counts[B_VSEEN + 1] = 2;  // both CTAs' V producers
     for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), counts[i]);
     fence_mbarrier_init_cluster();
     *abort_flag = 0;
@@ -363,10 +372,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true;
       bool have = g.init(p, w);
       uint32_t vc = 0;  // V slot counter
+      int gi = 0;
       while (have && ok) {
+        bool keep = true;
+        if constexpr (kSkip) {
+          // the pair's decision for this group: a skipped group's V is not loaded
+          ok = mbar_wait(bar(B_DECIDE + (gi & 1)), (gi >> 1) & 1, p.wait_limit_ns);
+          ok = __all_sync(0x3u, ok);
+          if (!ok) break;
+          keep = pair_keeps(gi);
+          __syncwarp(0x3u);
+          if (lane == 0) {  // both CTAs' publishers may now reuse this vote slot
+            mbar_arrive_local(bar(B_VSEEN + (gi & 1)));
+            mbar_arrive_cluster(map_to_cta(bar(B_VSEEN + (gi & 1)), rank ^ 1u));
+          }
+        }
+        ++gi;
         int rows[kGroupPages];
         for (int q = 0; q < kGroupPages; ++q) rows[q] = page_row(g.b, g.page + q, q < g.npages);
-        for (int q = 0; q < kGroupPages && ok; ++q) {
+        for (int q = 0; q < kGroupPages && ok && keep; ++q) {
           for (int nb = 0; nb < Wd::kNBlocks && ok; ++nb, ++vc) {
             const int slot = vc % C::kVSlots;
             if (vc >= (uint32_t)C::kVSlots)
@@ -442,18 +466,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t vc = 0;
       GroupCursor g;
       bool have = g.init(p, w);
+      int n_groups = 0, n_skipped = 0;
       for (int gi = 0; have && ok; ++gi) {
         ok = mbar_wait(bar(B_P_FULL), gi & 1, p.wait_limit_ns);
         if (ok && g.first && g.seg > 0) ok = mbar_wait(bar(B_O_FREE), (g.seg - 1) & 1, p.wait_limit_ns);
         if (!ok) break;
         MLA_TRACE_EV(w, 0, EV_PV_START, gi);
+        // threshold skipping: both CTAs' softmax warps read the pair's decision
+        // before arriving on B_P_FULL, so it is final here
+        bool keep = true;
+        if constexpr (kSkip) {
+          keep = pair_keeps(gi);
+          ++n_groups;
+          n_skipped += keep ? 0 : 1;
+        }
         // page-major: P of pages 0, 1 is released half way through
         for (int q = 0; q < kGroupPages && ok; ++q) {
           if (C::kSharedP && q == 2) {
             ok = mbar_wait(bar(B_P_FULL_HI), gi & 1, p.wait_limit_ns);  // pages 2, 3 in the shared P buffer
             if (!ok) break;
           }
-          for (int nb = 0; nb < Wd::kNBlocks && ok; ++nb, ++vc) {
+          for (int nb = 0; nb < Wd::kNBlocks && ok && keep; ++nb, ++vc) {
             const int shard = S == 2 ? nb : 0;
             const int slot = vc % C::kVSlots;
             ok = mbar_wait(bar(B_V_FULL + slot), (vc / C::kVSlots) & 1, p.wait_limit_ns);
@@ -481,6 +514,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_commit<2>(bar(B_FINAL_PV));
       if (!mbar_wait(bar(B_FINAL_PV), 0, p.wait_limit_ns)) ok = false;
       if (!ok) fail(MLA_ERR_DEVICE_TIMEOUT);
+      if constexpr (kSkip) {
+        atomicAdd(p.skip_stats, n_skipped);
+        atomicAdd(p.skip_stats + 1, n_groups);
+      }
     }
     __syncwarp();
   } else {
@@ -507,10 +544,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool have = g.init(p, w);
     int gi = 0;
     float m[S], l[S];
+    float mm = -INFINITY;  // threshold skipping: the row's true running max of the segment (log2 units)
     while (have) {
       if (g.first) {
 #pragma unroll
         for (int s = 0; s < S; ++s) { m[s] = -INFINITY; l[s] = 0.f; }
+        mm = -INFINITY;
       }
       const int sb = gi % C::kSBufs;
       float* xmax = xch + (gi & 1) * S * 128;      // this group's [S][128] row maxima
@@ -567,8 +606,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         named_sync();
         // row max over both token halves (the other half lives in lane lq ^ 64)
         const float mt = fmaxf(mt_own, xmax[s * 128 + (lq ^ 64)]);
+        // Threshold skipping (BLASST abstract on the kk6lht.com listing: a fixed
+        // threshold against the online softmax's running max marks negligible
+        // scores; their exp, value loads and PV are skipped). A row keeps the
+        // group if its maximum reaches its running max + skip_log2 (or it is the
+        // row's first visible group); the group is skipped when no row of the
+        // pair keeps it. Votes: a barrier reduction over this CTA's 128 softmax
+        // threads, exchanged with the peer by an async store on its barrier.
+        bool skip = false;
+        if constexpr (kSkip) {
+          const bool keep_row = row_real && mt != -INFINITY && (mm == -INFINITY || mt >= mm + p.skip_log2);
+          mm = fmaxf(mm, mt);
+          uint32_t any_keep;
+          asm volatile("{\n\t.reg .pred pk, pa;\n\tsetp.ne.u32 pk, %1, 0;\n\t"
+                       "barrier.cta.red.or.pred pa, 2, 128, pk;\n\tselp.u32 %0, 1, 0, pa;\n\t}"
+                       : "=r"(any_keep) : "r"((uint32_t)keep_row) : "memory");
+          const int par = gi & 1;
+          if (lq == 0) {
+            // the vote slot of group gi - 2 is free once both V producers read it
+            if (ok && gi >= 2) ok = mbar_wait(bar(B_VSEEN + par), ((gi - 2) >> 1) & 1, p.wait_limit_ns);
+            if (ok) {
+              votes[2 * par + rank] = any_keep;
+              const uint32_t slot = smem_u32(const_cast<uint32_t*>(votes + 2 * par + rank));
+              st_async_b32(map_to_cta(slot, rank ^ 1u), any_keep, map_to_cta(bar(B_DECIDE + par), rank ^ 1u));
+              mbar_arrive_expect_tx_local(bar(B_DECIDE + par), 4);
+            }
+          }
+          wait(B_DECIDE + par, (gi >> 1) & 1);
+          skip = ok && !pair_keeps(gi);
+        }
         float mu = m[s];
-        if (m[s] == -INFINITY || mt > m[s] + kRescaleThreshold) mu = fmaxf(mt, m[s]);
+        if (!skip && (m[s] == -INFINITY || mt > m[s] + kRescaleThreshold)) mu = fmaxf(mt, m[s]);
         float alpha = 1.f;
         const bool rescale = mu != m[s] && m[s] != -INFINITY;
         if (rescale) alpha = ex2_approx(m[s] - mu);
@@ -579,6 +647,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t pk[64];
         float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
         const float nmu = mu == -INFINITY ? 0.f : -mu;
+        if (!skip) {
 #pragma unroll
         for (int j = 0; j < 128; j += 4) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, nmu));
@@ -590,6 +659,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           __nv_bfloat162 h1 = __floats2bfloat162_rn(p2, p3);
           pk[j >> 1] = *reinterpret_cast<uint32_t*>(&h0);
           pk[(j >> 1) + 1] = *reinterpret_cast<uint32_t*>(&h1);
+        }
         }
         l[s] = l[s] * alpha + ((ps0 + ps1) + (ps2 + ps3));
         if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PASS2, gi);
@@ -635,7 +705,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             wait(B_P_FREE_LO, gi & 1);
           }
           if (lq == 0) MLA_TRACE_EV(w, rank, EV_PBUF_FREE, gi);
-          if (ok) {
+          if (ok && !skip) {
             write_p(gbase + L::p);
             fence_proxy_async_smem();
             tc_fence_before();
@@ -780,22 +850,28 @@ inline bool make_rows_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64
 }  // namespace tc
 
 namespace tc {
-template <int S, int R>
+template <int S, int R, bool kSkip = false>
 inline cudaError_t launch_decode_variant(const RunParams& p, const CUtensorMap& tm_kv, const CUtensorMap& tm_q,
                                          cudaStream_t stream, bool pdl) {
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_tc_kernel<S, R>), (int)Smem<S, R>::alloc);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_tc_kernel<S, R, kSkip>),
+                                    (int)Smem<S, R>::alloc);
   if (e != cudaSuccess) return e;
-  return launch_dependent_opt(pdl, decode_tc_kernel<S, R>, dim3(2 * p.W), dim3(kThreads), Smem<S, R>::alloc, stream,
-                              tm_kv, tm_q, p);
+  return launch_dependent_opt(pdl, decode_tc_kernel<S, R, kSkip>, dim3(2 * p.W), dim3(kThreads), Smem<S, R>::alloc,
+                              stream, tm_kv, tm_q, p);
 }
 }  // namespace tc
 
 // r = 512 with one or two latent shards, or r = 256 with one (a TPLA shard per GPU)
-inline cudaError_t launch_tc_decode(const RunParams& p, cudaStream_t stream, bool pdl = true) {
+// skip: the threshold-skipping variant (r = 512, one shard; p.skip_log2, p.skip_stats)
+inline cudaError_t launch_tc_decode(const RunParams& p, cudaStream_t stream, bool pdl = true, bool skip = false) {
   const uint64_t width = (uint64_t)p.r + p.dr;
   CUtensorMap tm_kv, tm_q;
   if (!tc::make_rows_map(&tm_kv, p.kv, (uint64_t)p.num_blocks * 64, width)) return cudaErrorInvalidValue;
   if (!tc::make_rows_map(&tm_q, p.q, (uint64_t)p.B * p.rows, width)) return cudaErrorInvalidValue;
+  if (skip) {
+    if (p.r != 512 || p.S != 1) return cudaErrorInvalidValue;
+    return tc::launch_decode_variant<1, 512, true>(p, tm_kv, tm_q, stream, pdl);
+  }
   if (p.r == 256 && p.S == 1) return tc::launch_decode_variant<1, 256>(p, tm_kv, tm_q, stream, pdl);
   if (p.r != 512) return cudaErrorInvalidValue;
   return p.S == 1 ? tc::launch_decode_variant<1, 512>(p, tm_kv, tm_q, stream, pdl)

@@ -18,6 +18,9 @@ synthetic because no trained weights are available):
                   [1024, 32768], 2 causal query tokens per sequence, paged
 * ``tpla_dsv3``   bf16, DeepSeek-V3 shape with the latent split into 2 shards
                   (TPLA), B=32, L=32768, paged
+* ``deepseek_v3_peaked`` the DeepSeek-V3 shape with peaked attention (a quarter
+                  of the tokens, in runs of 1024, relevant to every query;
+                  PEAK_* below): the threshold-skipping workload
 * ``deepseek_v3_fp8`` the DeepSeek-V3 shape over an FP8 latent cache: cKV as
                   E4M3 codes with one fp32 scale per token, the RoPE key bf16
                   stored divided by the token's scale; activations and weights
@@ -78,6 +81,7 @@ class Workload:
     dtype: str = "bf16"     # "bf16", "fp32" or "fp8" (FP8 cache, bf16 activations)
     paged: bool = True      # False: identity block table (contiguous cache)
     page_size: int = 64
+    peaked: bool = False    # True: clustered relevant keys (see PEAK_* below)
 
     @property
     def softmax_scale(self) -> float:
@@ -116,7 +120,30 @@ WORKLOADS = {
     "deepseek_v3_fp8": Workload("deepseek_v3_fp8", seed=5, batch=32, q_len=1, heads=128,
                                 latent_rank=512, rope_dim=64, nope_dim=128, v_dim=128,
                                 context=32768, dtype="fp8"),
+    "deepseek_v3_peaked": Workload("deepseek_v3_peaked", seed=7, batch=32, q_len=1, heads=128,
+                                   latent_rank=512, rope_dim=64, nope_dim=128, v_dim=128,
+                                   context=32768, peaked=True),
 }
+
+# Peaked attention (threshold-skipping workload). Synthetic N(0, 1) data gives
+# nearly flat attention; the pages' workloads are peaked. Here the tokens at
+# positions j with (j // PEAK_RUN) % PEAK_PERIOD == 0 (a quarter, in runs of
+# 1024) are relevant: their RoPE key is PEAK_KEEP * N(0, 1) + PEAK_GAIN * u,
+# every other token's RoPE key stays N(0, 1), and every query's RoPE part is
+# N(0, 1) + PEAK_GAIN * u, with u a seeded +-1 vector. A relevant key then
+# scores about scale * PEAK_GAIN^2 * d_rope (~10.4 at d_rope = 64, scale
+# 1/sqrt(192)) above an irrelevant one, for every head.
+PEAK_RUN, PEAK_PERIOD, PEAK_GAIN, PEAK_KEEP = 1024, 4, 1.5, 0.5
+_TAG_PEAK = 9
+
+
+def peak_direction(wl: Workload) -> torch.Tensor:
+    g = _gen(wl.seed, _TAG_PEAK)
+    return (torch.randint(0, 2, (wl.rope_dim,), generator=g) * 2 - 1).to(torch.float32)
+
+
+def relevant_tokens(length: int) -> torch.Tensor:
+    return (torch.arange(length) // PEAK_RUN) % PEAK_PERIOD == 0
 
 _TAG_LENS, _TAG_QN, _TAG_QR, _TAG_WUK, _TAG_WUV, _TAG_PERM = 1, 2, 3, 4, 5, 6
 _TAG_SEQ0 = 100
@@ -147,6 +174,9 @@ def draw_sequence_rows(wl: Workload, b: int, length: int) -> torch.Tensor:
     """[length, r + dr] latent rows of sequence b in the workload dtype."""
     g = _gen(wl.seed, _TAG_SEQ0 + b)
     x = torch.randn((length, wl.row_width), generator=g, dtype=torch.float32)
+    if wl.peaked:
+        rel = relevant_tokens(length)
+        x[rel, wl.latent_rank:] = PEAK_KEEP * x[rel, wl.latent_rank:] + PEAK_GAIN * peak_direction(wl)
     return x.to(wl.torch_dtype)
 
 
@@ -169,7 +199,10 @@ def generate(wl: Workload, seq_lens: Optional[Sequence[int]] = None,
                             wl.heads, wl.q_len)
     out = {"seq_lens": lens}
     out["q_nope"] = torch.randn((B, Lq, H, dn), generator=_gen(wl.seed, _TAG_QN)).to(dt)
-    out["q_rope"] = torch.randn((B, Lq, H, dr), generator=_gen(wl.seed, _TAG_QR)).to(dt)
+    qr = torch.randn((B, Lq, H, dr), generator=_gen(wl.seed, _TAG_QR))
+    if wl.peaked:
+        qr = qr + PEAK_GAIN * peak_direction(wl)
+    out["q_rope"] = qr.to(dt)
     wstd = 1.0 / math.sqrt(r)
     out["w_uk"] = (torch.randn((H, dn, r), generator=_gen(wl.seed, _TAG_WUK)) * wstd).to(dt)
     out["w_uv"] = (torch.randn((H, r, dv), generator=_gen(wl.seed, _TAG_WUV)) * wstd).to(dt)

@@ -244,3 +244,22 @@ def test_timeout_selftest_argument_checks(kw, kernel, limit, status):
         assert e.value.status == status
     finally:
         L.mla_plan_destroy(plan)
+
+
+@pytest.mark.parametrize("kw,thr,status", [
+    (dict(), 0.5, L.MLA_ERR_INVALID_ARG),            # a threshold above the running max
+    (dict(), float("nan"), L.MLA_ERR_INVALID_ARG),
+    (dict(dtype="fp8"), -6.0, L.MLA_ERR_UNSUPPORTED),
+    (dict(latent_shards=2), -6.0, L.MLA_ERR_UNSUPPORTED),
+])
+def test_blasst_argument_checks(kw, thr, status):
+    """Threshold skipping takes bf16, one latent shard and a threshold <= 0;
+    the checks come before any device work."""
+    plan, ws = L.mla_decode_plan_ex(_dims(**kw), [4000, 65], num_sms=148, kernel=L.MLA_KERNEL_AUTO)
+    try:
+        fake = 1 << 20  # never dereferenced
+        with pytest.raises(L.MlaError) as e:
+            L.mla_decode_run_blasst(plan, fake, fake, fake, 1, fake, 64, fake, fake, fake, fake, fake, ws, thr)
+        assert e.value.status == status
+    finally:
+        L.mla_plan_destroy(plan)
