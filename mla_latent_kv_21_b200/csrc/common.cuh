@@ -67,13 +67,15 @@ MLA_HD int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 //   [0]            int32 status word (first device-side error, sticky)
 //   [4]            int32 lengths_ok (written by the first kernel of a run)
 //   cum            int64 [B + 1] page prefix sums of this run's seq_lens
+//   done           int32 [B] segment halves of sequence b written this run
+//                  (each CTA of a pair adds 1 per segment once its rows are out)
 //   q              [B * Lq * H, r + d_rope] absorbed query rows (dims.dtype)
 //   o_part         [slots, rows, r]  per-segment O_lat / l: fp32 on the SIMT
 //                  path, fp16 on the tensor-core paths (room for fp32 either way)
 //   lse_part       fp32 [slots, rows, S]  per-segment log2-sum-exp per shard
 // ---------------------------------------------------------------------------
 struct WorkspaceLayout {
-  size_t cum, q, o_part, lse_part, total;
+  size_t cum, done, q, o_part, lse_part, total;
 };
 
 MLA_HD size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -85,6 +87,8 @@ inline WorkspaceLayout workspace_layout(int64_t B, int64_t Lq, int64_t H, int64_
   size_t off = 1024;
   L.cum = off;
   off = align_up(off + sizeof(int64_t) * (B + 1), 1024);
+  L.done = off;
+  off = align_up(off + sizeof(int32_t) * B, 1024);
   L.q = off;
   off = align_up(off + (size_t)(B * Lq * H) * (r + dr) * elt_bytes, 1024);
   L.o_part = off;
@@ -117,6 +121,7 @@ struct RunParams {
   int32_t* status;
   int32_t* lengths_ok;
   int64_t* cum;
+  int32_t* seg_done;       // [B] zeroed by the absorb kernel, counted up by the decode kernels
   void* q;                 // absorbed query rows
   float* o_part;           // fp32 (SIMT kernels) or fp16 (tensor-core kernels)
   float* lse_part;
@@ -144,6 +149,19 @@ bool plan_is_fp8(const mla_plan* plan);
 
 __device__ __forceinline__ void record_error(int32_t* status, int32_t code) {
   atomicCAS(status, 0, code);
+}
+
+// A CTA of a decode pair has written its rows of a segment's partials: every
+// writing thread fenced its stores before the CTA barrier that precedes this
+// call, so the release-ordered add publishes them at GPU scope.
+__device__ __forceinline__ void publish_segment_half(int32_t* done) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" :: "l"(done) : "memory");
+}
+
+__device__ __forceinline__ int32_t load_acquire_gpu(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ float to_float(float x) { return x; }

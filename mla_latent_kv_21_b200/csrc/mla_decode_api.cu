@@ -244,6 +244,7 @@ mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, c
   p.status = reinterpret_cast<int32_t*>(ws);
   p.lengths_ok = reinterpret_cast<int32_t*>(ws + 4);
   p.cum = reinterpret_cast<int64_t*>(ws + plan->layout.cum);
+  p.seg_done = reinterpret_cast<int32_t*>(ws + plan->layout.done);
   p.q = ws + plan->layout.q;
   p.o_part = reinterpret_cast<float*>(ws + plan->layout.o_part);
   p.lse_part = reinterpret_cast<float*>(ws + plan->layout.lse_part);

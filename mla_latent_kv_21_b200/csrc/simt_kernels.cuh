@@ -56,6 +56,7 @@ __device__ void scan_lengths(const RunParams& p) {
   int64_t acc = part[tid];
   for (int b = b0; b < b1; ++b) {
     p.cum[b] = acc;
+    if (p.seg_done) p.seg_done[b] = 0;
     const int64_t L = p.seq_lens[b];
     acc += ceil_div64(L > 0 ? L : 0, p.P);
   }

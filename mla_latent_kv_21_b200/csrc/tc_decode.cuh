@@ -794,8 +794,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             __syncwarp();
           }
           tc_fence_before();
+          __threadfence();  // this thread's partial rows, before the CTA's segment-done count
         }
         named_sync();  // xl and the O reads of all four warps are done
+        if (ok && lq == 0) publish_segment_half(p.seg_done + g.b);
         if (lq == 0) MLA_TRACE_EV(w, rank, EV_LD0, gi);
         __syncwarp();
         if (ok && lane == 0) arrive_leader(B_O_FREE);

@@ -129,13 +129,30 @@ __global__ void __launch_bounds__(kThreads, 4)
       record_error(p.status, MLA_ERR_DEVICE_TIMEOUT);
     }
   }
-  // q_rope columns of the packed query rows (the tile-0 CTA of each head)
+  // q_rope columns of the packed query rows (the tile-0 CTA of each head), in
+  // 16-byte pieces (d_rope = 64: 8 per row, at most 4 per thread for 128 rows),
+  // every load issued before the first store
   if (mt == 0) {
-    const __nv_bfloat16* q_rope = static_cast<const __nv_bfloat16*>(p.q_rope);
-    __nv_bfloat16* q = static_cast<__nv_bfloat16*>(p.q);
-    for (int idx = threadIdx.x; idx < nrows * p.dr; idx += blockDim.x) {
-      const int i = idx / p.dr, e = idx % p.dr, bt = row0 + i;
-      q[((int64_t)bt * p.H + h) * (p.r + p.dr) + p.r + e] = q_rope[((int64_t)bt * p.H + h) * p.dr + e];
+    const uint4* q_rope = static_cast<const uint4*>(p.q_rope);
+    uint4* q = static_cast<uint4*>(p.q);
+    constexpr int kPer = (kAbsorbMaxN * 8 + kThreads - 1) / kThreads;
+    const int total = nrows * 8;
+    uint4 v[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int idx = threadIdx.x + k * kThreads;
+      if (idx < total) {
+        const int64_t row = (int64_t)(row0 + idx / 8) * p.H + h;
+        v[k] = __ldg(q_rope + row * 8 + (idx % 8));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int idx = threadIdx.x + k * kThreads;
+      if (idx < total) {
+        const int64_t row = (int64_t)(row0 + idx / 8) * p.H + h;
+        q[row * ((p.r + p.dr) / 8) + p.r / 8 + (idx % 8)] = v[k];  // row of (r + d_rope) bf16 = 72 pieces
+      }
     }
   }
   __syncwarp();
@@ -246,7 +263,12 @@ __global__ void __launch_bounds__(kCombineThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tslot;
   grid_launch_dependents();
-  grid_dependency_wait();  // the partials of the decode kernel
+  // No grid-wide wait for the decode kernel: this grid starts once every decode
+  // CTA has passed its setup (all of them resident), and each merge item waits
+  // below for its own sequence's segments only, so the sequences that finish
+  // early are merged while the last decode pairs still run. The prefix sums and
+  // the length flag come from the absorb kernel, complete before the decode
+  // kernel started.
   const bool run = *p.lengths_ok != 0;
   if (run) {
     // ---- merge: one item = one row x 32 latent columns (64 bytes of each fp16
@@ -267,6 +289,20 @@ __global__ void __launch_bounds__(kCombineThreads, 1)
         const int sh = c0 / (p.r / S);
         const int64_t lo = page_owner(p.cum[b], b, Gv, p.W) + b;
         const int64_t hi = page_owner(p.cum[b + 1] - 1, b, Gv, p.W) + b;
+        // both CTAs of each of the sequence's segments publish their rows (bounded wait)
+        const int32_t want = 2 * (int32_t)(hi - lo + 1);
+        if (load_acquire_gpu(p.seg_done + b) < want) {
+          const uint64_t t0 = ptx::globaltimer_ns();
+          bool waited = true;
+          while (load_acquire_gpu(p.seg_done + b) < want) {
+            if (ptx::globaltimer_ns() - t0 > p.wait_limit_ns) {
+              waited = false;
+              break;
+            }
+            __nanosleep(128);
+          }
+          if (!waited) record_error(p.status, MLA_ERR_DEVICE_TIMEOUT);
+        }
         const float* lse = p.lse_part + (int64_t)row * S + sh;
         const __half* op = opart + (int64_t)row * p.r + c0;
         // one round of loads per 4 segments; the running maximum moves as the
