@@ -27,6 +27,10 @@
 //       pages 2-3 once the PV MMAs are done with the first half.
 //   TPLA (S = 2 shards): one S tile per shard (latent chunks 0-3 or 4-7, each
 //       with the RoPE chunk), one softmax per shard, PV N block nb = shard nb.
+//       The QK chunk order puts the RoPE chunk between the shards, so shard
+//       0's tile is complete (and released) on its own; each shard has its
+//       own 16 KB P buffer with the one-shard hand-off, and V items run
+//       shard by shard within each page half.
 //
 // QK and PV are issued by two different threads of the leader CTA, so that the
 // QK stream (HBM) and the V stream (L2) drain independently; they touch
@@ -70,6 +74,16 @@ struct Width {
   static constexpr uint32_t kQBytes = kChunks * kQChunkBytes;
   static constexpr uint32_t kOCols = R / 2;
 };
+// Chunk order within a group. One shard: latent chunks 0..R/64-1, then the
+// RoPE chunk. Two shards (r = 512): shard 0's latent chunks 0-3, the RoPE
+// chunk (added to both shards' scores), then shard 1's chunks 4-7, so shard
+// 0's scores are complete after five chunks and the softmax starts on them
+// while shard 1's QK is still running.
+template <int S>
+__device__ __forceinline__ int chunk_at(int pos) {
+  if constexpr (S == 2) return pos < 4 ? pos : (pos == 4 ? 8 : pos - 1);
+  return pos;
+}
 constexpr uint32_t kSlotBytes = 16384;       // QK slot: 128 tokens x 64 cols; V slot: 64 tokens x 128 cols
 constexpr uint32_t kPChunkBytes = 64 * 128;  // 64 rows x 64 tokens bf16
 constexpr uint32_t kPBytes = 4 * kPChunkBytes;  // 64 rows x 256 tokens
@@ -87,16 +101,23 @@ constexpr int kIssueLanes = 2;
 #ifndef MLA_V_SLOTS
 #define MLA_V_SLOTS 4
 #endif
+#ifndef MLA_QK_SLOTS_2SHARD
+#define MLA_QK_SLOTS_2SHARD 3
+#endif
+#ifndef MLA_V_SLOTS_2SHARD
+#define MLA_V_SLOTS_2SHARD 4
+#endif
 template <int S, int R = 512>
 struct Cfg {
-  static constexpr int kQkSlots = S == 1 ? MLA_QK_SLOTS : 3;
-  static constexpr int kVSlots = S == 1 ? MLA_V_SLOTS : 2;
+  static constexpr int kQkSlots = S == 1 ? MLA_QK_SLOTS : MLA_QK_SLOTS_2SHARD;
+  static constexpr int kVSlots = S == 1 ? MLA_V_SLOTS : MLA_V_SLOTS_2SHARD;
   static constexpr int kSBufs = S == 1 ? 2 : 1;   // S tiles in tensor memory (128 columns each per shard)
-  // One shard: a single 16 KB P buffer holds group pages 0, 1 and then 2, 3
-  // (the second half is written once PV is done with the first), which frees
-  // 16 KB for a fourth QK ring slot. Two shards keep P for all four pages.
-  static constexpr bool kSharedP = S == 1;
-  static constexpr uint32_t kPRegion = kSharedP ? kPBytes / 2 : S * kPBytes;
+  // P per shard: one 16 KB buffer holds group pages 0, 1 and then 2, 3 (the
+  // second half is written once PV is done with the first). Against P for all
+  // four pages this frees 16 KB per shard for the TMA rings, whose depth sets
+  // the streaming rate.
+  static constexpr uint32_t kPShard = kPBytes / 2;
+  static constexpr uint32_t kPRegion = S * kPShard;
 };
 
 template <int S, int R = 512>
@@ -120,24 +141,50 @@ enum : int {
   B_Q_FULL = 0,       // (unused: the query arrives chunk by chunk, B_QC_FULL)
   B_QK_FULL = 1,      // [6] leader, count 2 (+tx)
   B_V_FULL = 7,       // [6] leader, count 2 (+tx)
-  B_S_FREE = 13,      // [2] leader, count 8 (4 softmax warps x 2 CTAs)
-  B_P_FULL = 15,      // leader, count 8: P written (shared P: pages 0, 1 written and O rescaled)
+  B_S_FREE = 13,      // [2] leader, count 8 (4 softmax warps x 2 CTAs): by S buffer (one shard) or by shard
+  B_P_FULL = 15,      // leader, count 8: P pages 0, 1 written (2 warps x 2 CTAs) and O rescaled (all 8)
   B_O_FREE = 16,      // leader, count 8
   B_QK_FREE = 17,     // [6] both, count 1 (MMA commit)
   B_V_FREE = 23,      // [6] both, count 1
-  B_S_FULL = 29,      // [2] both, count 1
+  B_S_FULL = 29,      // [2] both, count 1: by S buffer (one shard) or by shard (two)
   B_PV_DONE = 31,     // both, count 1
   B_FINAL_QK = 32,    // leader, count 1
   B_FINAL_PV = 33,    // leader, count 1
   B_P_FREE_LO = 34,   // both, count 1: PV is done with P of group pages 0, 1
   B_P_FREE_HI = 35,   // both, count 1: PV is done with P of group pages 2, 3
   B_QC_FULL = 36,     // [9] leader, count 2 (+tx): query chunk k of the current segment
-  B_P_FULL_HI = 45,   // leader, count 4 (shared P: pages 2, 3 written by 2 warps x 2 CTAs)
+  B_P_FULL_HI = 45,   // leader, count 4: P pages 2, 3 written by 2 warps x 2 CTAs
   // threshold skipping (kSkip): the pair's keep / skip decision of group gi
   B_DECIDE = 46,      // [2] both, count 1 (+4 tx bytes: the peer's vote), by group parity
   B_VSEEN = 48,       // [2] both, count 1: the V producer has read the decision of group gi
-  B_COUNT = 50
+  // two shards: shard 1's copies of B_P_FULL, B_P_FULL_HI, B_P_FREE_LO, B_P_FREE_HI
+  B_P_FULL_1 = 50,
+  B_P_FULL_HI_1 = 51,
+  B_P_FREE_LO_1 = 52,
+  B_P_FREE_HI_1 = 53,
+  B_COUNT = 54
 };
+// the P hand-off barriers of shard s
+__host__ __device__ constexpr int bar_p_full(int s) { return s ? B_P_FULL_1 : B_P_FULL; }
+__host__ __device__ constexpr int bar_p_full_hi(int s) { return s ? B_P_FULL_HI_1 : B_P_FULL_HI; }
+__host__ __device__ constexpr int bar_p_free_lo(int s) { return s ? B_P_FREE_LO_1 : B_P_FREE_LO; }
+__host__ __device__ constexpr int bar_p_free_hi(int s) { return s ? B_P_FREE_HI_1 : B_P_FREE_HI; }
+static_assert(B_COUNT <= 56, "barrier array");
+
+// V ring order within a group: item i -> (page q, N block nb). One shard:
+// page-major. Two shards (N block nb = shard nb): pages 0, 1 of shard 0,
+// pages 0, 1 of shard 1, then pages 2, 3 of each, so that PV releases each
+// shard's first P half as early as the one-shard order does.
+template <int S, int NB>
+__device__ __forceinline__ void v_item(int i, int& q, int& nb) {
+  if constexpr (S == 2) {
+    nb = (i >> 1) & 1;
+    q = 2 * (i >> 2) + (i & 1);
+  } else {
+    q = i / NB;
+    nb = i % NB;
+  }
+}
 
 // Optional event trace (compile with -DMLA_TRACE): SM clock of per-group events
 // of the first kTraceWorkers workers, read back with mla_debug_trace_read().
@@ -240,7 +287,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   using C = Cfg<S, R>;
   using Wd = Width<R>;
   static_assert(S == 1 || R == 512, "two shards in one launch split r = 512");
-  static_assert(!kSkip || (S == 1 && C::kSharedP), "threshold skipping: one latent shard");
+  static_assert(!kSkip || S == 1, "threshold skipping: one latent shard");
   constexpr int kChunks = Wd::kChunks;
   extern __shared__ uint8_t smem_raw[];
   MLA_TRACE_CTA(0);
@@ -281,8 +328,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 6; ++i) counts[B_QK_FULL + i] = 2;
     for (int i = 0; i < 6; ++i) counts[B_V_FULL + i] = 2;
     counts[B_S_FREE] = counts[B_S_FREE + 1] = 8;
-    counts[B_P_FULL] = 8;
-    counts[B_P_FULL_HI] = 4;
+    counts[B_P_FULL] = counts[B_P_FULL_1] = 8;
+    counts[B_P_FULL_HI] = counts[B_P_FULL_HI_1] = 4;
     counts[B_O_FREE] = 8;
     counts[B_VSEEN] = counts[B_VSEEN + 1] = 2;  // both CTAs' V producers
     for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), counts[i]);
@@ -341,14 +388,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int pg = 2 * (int)rank + lane;            // this lane's page within the group
         const int y = page_row(g.b, g.page + pg, pg < g.npages);
         if (lane == 0) MLA_TRACE_EV(w, rank, EV_LOAD, gi);
-        for (int kc = 0; kc < kChunks && ok; ++kc, ++cc) {
+        for (int pos = 0; pos < kChunks && ok; ++pos, ++cc) {
+          const int kc = chunk_at<S>(pos);
           const int slot = cc % C::kQkSlots;
           if (cc >= (uint32_t)C::kQkSlots)
             ok = mbar_wait(bar(B_QK_FREE + slot), ((cc / C::kQkSlots) - 1) & 1, p.wait_limit_ns);
           if (!ok) break;
           if (g.first && lane == 1) {
             // New segment: reload query chunk kc. Its last reader, chunk kc of
-            // the previous group (9 items back), is done: the QK issuer
+            // the previous group (kChunks items back), is done: the QK issuer
             // consumes items in order and item cc - kQkSlots has been released.
             expect_leader(B_QC_FULL + kc, kQChunkBytes);
             tma_load_2d_pair(base + L::q + kc * kQChunkBytes, &tm_q, 64 * kc, yq,
@@ -390,18 +438,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ++gi;
         int rows[kGroupPages];
         for (int q = 0; q < kGroupPages; ++q) rows[q] = page_row(g.b, g.page + q, q < g.npages);
-        for (int q = 0; q < kGroupPages && ok && keep; ++q) {
-          for (int nb = 0; nb < Wd::kNBlocks && ok; ++nb, ++vc) {
-            const int slot = vc % C::kVSlots;
-            if (vc >= (uint32_t)C::kVSlots)
-              ok = mbar_wait(bar(B_V_FREE + slot), ((vc / C::kVSlots) - 1) & 1, p.wait_limit_ns);
-            if (!ok) break;
-            if (lane == 0) expect_leader(B_V_FULL + slot, kSlotBytes);
-            const int chunk = 4 * nb + 2 * (int)rank + lane;
-            tma_load_2d_pair(base + L::v + slot * kSlotBytes + lane * (kSlotBytes / 2), &tm_kv, 64 * chunk,
-                             rows[q], leader_bar(B_V_FULL + slot));
-            if (lane == 0) MLA_TRACE_CHUNK(w, rank, 2, vc);
-          }
+        for (int i = 0; i < kGroupPages * Wd::kNBlocks && ok && keep; ++i, ++vc) {
+          int q, nb;
+          v_item<S, Wd::kNBlocks>(i, q, nb);
+          const int slot = vc % C::kVSlots;
+          if (vc >= (uint32_t)C::kVSlots)
+            ok = mbar_wait(bar(B_V_FREE + slot), ((vc / C::kVSlots) - 1) & 1, p.wait_limit_ns);
+          if (!ok) break;
+          if (lane == 0) expect_leader(B_V_FULL + slot, kSlotBytes);
+          const int chunk = 4 * nb + 2 * (int)rank + lane;
+          tma_load_2d_pair(base + L::v + slot * kSlotBytes + lane * (kSlotBytes / 2), &tm_kv, 64 * chunk,
+                           rows[q], leader_bar(B_V_FULL + slot));
+          if (lane == 0) MLA_TRACE_CHUNK(w, rank, 2, vc);
         }
         if (ok) have = g.next(p);
       }
@@ -421,12 +469,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       GroupCursor g;
       bool have = g.init(p, w);
       for (int gi = 0; have && ok; ++gi) {
+        // one shard: S buffer sb must be free; two shards (one buffer, a
+        // 128-column tile per shard): shard 0's tile now, shard 1's at the RoPE chunk
         const int sb = gi % C::kSBufs;
         if (ok && gi >= C::kSBufs) ok = mbar_wait(bar(B_S_FREE + sb), ((gi / C::kSBufs) - 1) & 1, p.wait_limit_ns);
         if (!ok) break;
         MLA_TRACE_EV(w, 0, EV_QK_START, gi);
         const uint32_t s_tmem = tbase + sb * 128 * S;
-        for (int kc = 0; kc < kChunks && ok; ++kc, ++cc) {
+        for (int pos = 0; pos < kChunks && ok; ++pos, ++cc) {
+          const int kc = chunk_at<S>(pos);
           const int slot = cc % C::kQkSlots;
           if (g.first) ok = mbar_wait(bar(B_QC_FULL + kc), g.seg & 1, p.wait_limit_ns);  // this segment's query chunk
           ok = ok && mbar_wait(bar(B_QK_FULL + slot), (cc / C::kQkSlots) & 1, p.wait_limit_ns);
@@ -435,20 +486,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint64_t ad = q_desc0 + (uint64_t)(kc * (kQChunkBytes >> 4));
           const uint64_t bd = qk_desc0 + (uint64_t)((slot * kSlotBytes) >> 4);
-#pragma unroll
-          for (int shard = 0; shard < S; ++shard) {
-            if (S == 2 && kc < 8 && (kc >> 2) != shard) continue;
-            const bool first_k = (S == 2) ? (kc == 4 * shard) : (kc == 0);
+          auto qk_mma = [&](int shard, bool first_k) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
               mma_f16<2>(s_tmem + 128 * shard, ad + (uint64_t)(2 * ks), bd + (uint64_t)(2 * ks),
                          idesc_qk, (first_k && ks == 0) ? 0u : 1u);
+          };
+          if constexpr (S == 1) {
+            qk_mma(0, kc == 0);
+          } else {
+            // shard 0: chunks 0-3 and the RoPE chunk, which completes it
+            if (kc < 4 || kc == 8) qk_mma(0, kc == 0);
+            if (kc == 8) {
+              commit_both(B_S_FULL + 0);
+              if (gi >= 1) ok = mbar_wait(bar(B_S_FREE + 1), (gi - 1) & 1, p.wait_limit_ns);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            // shard 1: the RoPE chunk first, then chunks 4-7
+            if (kc >= 4) qk_mma(1, kc == 8);
           }
           commit_both(B_QK_FREE + slot);
         }
         if (!ok) break;
         MLA_TRACE_EV(w, 0, EV_QK_END, gi);
-        commit_both(B_S_FULL + sb);
+        commit_both(B_S_FULL + (S == 2 ? 1 : sb));
         have = g.next(p);
       }
       tc_commit<2>(bar(B_FINAL_QK));
@@ -480,21 +542,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ++n_groups;
           n_skipped += keep ? 0 : 1;
         }
-        // page-major: P of pages 0, 1 is released half way through
-        for (int q = 0; q < kGroupPages && ok; ++q) {
-          if (C::kSharedP && q == 2) {
-            ok = mbar_wait(bar(B_P_FULL_HI), gi & 1, p.wait_limit_ns);  // pages 2, 3 in the shared P buffer
-            if (!ok) break;
+        // A shard's P buffer holds pages 0, 1, then pages 2, 3: PV waits for
+        // each half as it is written and releases it once its MMAs are issued
+        // (the commit completes when they are done). Items in V ring order.
+        if constexpr (S == 1) {
+          // page-major, both N blocks of a page (kept in this form: one loop
+          // over the items in ring order measured ~10% slower per step)
+          for (int q = 0; q < kGroupPages && ok; ++q) {
+            if (q == 2) {
+              ok = mbar_wait(bar(B_P_FULL_HI), gi & 1, p.wait_limit_ns);
+              if (!ok) break;
+            }
+            for (int nb = 0; nb < Wd::kNBlocks && ok && keep; ++nb, ++vc) {
+              const int slot = vc % C::kVSlots;
+              ok = mbar_wait(bar(B_V_FULL + slot), (vc / C::kVSlots) & 1, p.wait_limit_ns);
+              if (!ok) break;
+              MLA_TRACE_CHUNK(w, 0, 3, vc);
+              tc_fence_after();
+              const uint64_t pd = p_desc0 + (uint64_t)(((q & 1) * kPChunkBytes) >> 4);
+              const uint64_t vd = v_desc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                mma_f16<2>(tbase + kTmemO + 128 * nb, pd + (uint64_t)(2 * ks),
+                           vd + (uint64_t)(128 * ks), idesc_pv,
+                           (g.first && q == 0 && ks == 0) ? 0u : 1u);
+              commit_both(B_V_FREE + slot);
+            }
+            if (q == 1) commit_both(B_P_FREE_LO);
           }
-          for (int nb = 0; nb < Wd::kNBlocks && ok && keep; ++nb, ++vc) {
-            const int shard = S == 2 ? nb : 0;
+          if (ok) commit_both(B_P_FREE_HI);
+        } else {
+          auto pv_item = [&](int q, int shard) {  // N block nb = shard
+            const int nb = shard;
             const int slot = vc % C::kVSlots;
             ok = mbar_wait(bar(B_V_FULL + slot), (vc / C::kVSlots) & 1, p.wait_limit_ns);
-            if (!ok) break;
+            if (!ok) return;
             MLA_TRACE_CHUNK(w, 0, 3, vc);
             tc_fence_after();
-            const int pchunk = C::kSharedP ? (q & 1) : q;
-            const uint64_t pd = p_desc0 + (uint64_t)((shard * kPBytes + pchunk * kPChunkBytes) >> 4);
+            const uint64_t pd = p_desc0 + (uint64_t)((shard * C::kPShard + (q & 1) * kPChunkBytes) >> 4);
             const uint64_t vd = v_desc0 + (uint64_t)((slot * kSlotBytes) >> 4);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
@@ -502,12 +587,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                          vd + (uint64_t)(128 * ks), idesc_pv,
                          (g.first && q == 0 && ks == 0) ? 0u : 1u);
             commit_both(B_V_FREE + slot);
+            ++vc;
+          };
+          // page half, then shard (= N block), then the half's two pages
+          for (int hf = 0; hf < 2 && ok; ++hf) {
+            for (int sh = 0; sh < 2 && ok; ++sh) {
+              if (hf + sh > 0) {
+                ok = mbar_wait(bar(hf ? bar_p_full_hi(sh) : bar_p_full(sh)), gi & 1, p.wait_limit_ns);
+                if (!ok) break;
+              }
+              for (int qq = 0; qq < 2 && ok; ++qq) pv_item(2 * hf + qq, sh);
+              if (ok) commit_both(hf ? bar_p_free_hi(sh) : bar_p_free_lo(sh));
+            }
           }
-          if (q == 1) commit_both(B_P_FREE_LO);
         }
         if (!ok) break;
         MLA_TRACE_EV(w, 0, EV_PV_END, gi);
-        commit_both(B_P_FREE_HI);
         commit_both(B_PV_DONE);
         have = g.next(p);
       }
@@ -565,11 +660,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       nv = nv < 0 ? 0 : (nv > 128 ? 128 : nv);
       const int nvis = (int)nv;
 
-      wait(B_S_FULL + sb, (gi / C::kSBufs) & 1);
-      if (lq == 0) MLA_TRACE_EV(w, rank, EV_S_READY, gi);
-      if (ok) tc_fence_after();
+      if constexpr (S == 1) {
+        wait(B_S_FULL + sb, (gi / C::kSBufs) & 1);
+        if (lq == 0) MLA_TRACE_EV(w, rank, EV_S_READY, gi);
+        if (ok) tc_fence_after();
+      }
 #pragma unroll 1
       for (int s = 0; s < S; ++s) {
+        if constexpr (S == 2) {
+          // two shards: each tile is complete (and released) on its own
+          wait(B_S_FULL + s, gi & 1);
+          if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_S_READY, gi);
+          if (ok) tc_fence_after();
+        }
         // one pass over tensor memory: the thread's 128 scores of shard s
         uint32_t r[128];
         if (ok) {
@@ -579,11 +682,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       *reinterpret_cast<uint32_t(*)[32]>(r + c0));
           tmem_wait_ld();
         }
-        if (s == S - 1) {
-          // every score of this S buffer is in registers: QK may reuse it
+        if (S == 2 || s == S - 1) {
+          // every score of this S buffer (two shards: of this shard's tile)
+          // is in registers: QK may reuse it
           if (ok) tc_fence_before();
           __syncwarp();
-          if (ok && lane == 0 && !p.withhold_s_free) arrive_leader(B_S_FREE + sb);
+          if (ok && lane == 0 && !p.withhold_s_free) arrive_leader(B_S_FREE + (S == 2 ? s : sb));
         }
         // masked keys (past the group or the causal limit) become -inf: they
         // drop out of the max and 2^-inf = 0 in the sum and in P
@@ -689,48 +793,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                              pk[32 * t + 4 * u + 2], pk[32 * t + 4 * u + 3]);
           }
         };
-        if constexpr (C::kSharedP) {
-          // O is rescaled (after the previous group's PV) before this group's
-          // PV adds to it; both halves signal that through B_P_FULL.
-          if (!g.first && __any_sync(0xffffffffu, rescale)) wait(B_PV_DONE, (gi - 1) & 1);
-          if (ok && !g.first && __any_sync(0xffffffffu, rescale)) rescale_o(0, Wd::kOCols);
-          if (half == 0) {
-            // pages 0, 1: the previous group's PV must be done with pages 2, 3
-            if (gi >= 1) wait(B_P_FREE_HI, (gi - 1) & 1);
-          } else {
-            if (ok) tc_fence_before();
-            __syncwarp();
-            if (ok && lane == 0) arrive_leader(B_P_FULL);
-            // pages 2, 3 go where pages 0, 1 were, once this group's PV is done with them
-            wait(B_P_FREE_LO, gi & 1);
-          }
-          if (lq == 0) MLA_TRACE_EV(w, rank, EV_PBUF_FREE, gi);
-          if (ok && !skip) {
-            write_p(gbase + L::p);
-            fence_proxy_async_smem();
-            tc_fence_before();
-          }
-          __syncwarp();
-          if (ok && lane == 0) arrive_leader(half == 0 ? B_P_FULL : B_P_FULL_HI);
+        // Shard s's P buffer: pages 0, 1 (this half 0 thread's tokens) go in
+        // once the previous group's PV is done with pages 2, 3; pages 2, 3
+        // (half 1) replace them once this group's PV is done with pages 0, 1.
+        // Shard s's O columns are rescaled (after the previous group's PV)
+        // before this group's PV adds to them; both halves signal that
+        // through the shard's P_FULL barrier.
+        if (!g.first && __any_sync(0xffffffffu, rescale)) wait(B_PV_DONE, (gi - 1) & 1);
+        if (ok && !g.first && __any_sync(0xffffffffu, rescale))
+          rescale_o((Wd::kOCols / S) * s, Wd::kOCols / S);
+        if (half == 0) {
+          if (gi >= 1) wait(bar_p_free_hi(s), (gi - 1) & 1);
         } else {
-          // this warp's P chunks (2 half, 2 half + 1): the previous group's PV
-          // must be done with them
-          if (s == 0 && gi >= 1) wait(half ? B_P_FREE_HI : B_P_FREE_LO, (gi - 1) & 1);
-          if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PBUF_FREE, gi);
-          // rescale this shard's O columns (128 per shard) once the previous
-          // group's PV is complete
-          if (!g.first && __any_sync(0xffffffffu, rescale)) wait(B_PV_DONE, (gi - 1) & 1);
-          if (ok && !g.first && __any_sync(0xffffffffu, rescale)) rescale_o((256 / S) * s, 256 / S);
-          if (ok) write_p(gbase + L::p + s * kPBytes + 2 * half * kPChunkBytes);
+          if (ok) tc_fence_before();
+          __syncwarp();
+          if (ok && lane == 0) arrive_leader(bar_p_full(s));
+          wait(bar_p_free_lo(s), gi & 1);
         }
-      }
-      if constexpr (!C::kSharedP) {
-        if (ok) {
+        if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PBUF_FREE, gi);
+        if (ok && !skip) {
+          write_p(gbase + L::p + s * C::kPShard);
           fence_proxy_async_smem();
           tc_fence_before();
         }
         __syncwarp();
-        if (ok && lane == 0) arrive_leader(B_P_FULL);
+        if (ok && lane == 0) arrive_leader(half == 0 ? bar_p_full(s) : bar_p_full_hi(s));
       }
       if (lq == 0) MLA_TRACE_EV(w, rank, EV_P_DONE, gi);
 
