@@ -29,8 +29,10 @@
 //       with the RoPE chunk), one softmax per shard, PV N block nb = shard nb.
 //       The QK chunk order puts the RoPE chunk between the shards, so shard
 //       0's tile is complete (and released) on its own; each shard has its
-//       own 16 KB P buffer with the one-shard hand-off, and V items run
-//       shard by shard within each page half.
+//       own softmax warpgroup (384 threads per CTA, so 168 registers: the
+//       scores are read from tensor memory twice, for the max and for P) and
+//       its own 16 KB P buffer with the one-shard hand-off; V items run shard
+//       by shard within each page half.
 //
 // QK and PV are issued by two different threads of the leader CTA, so that the
 // QK stream (HBM) and the V stream (L2) drain independently; they touch
@@ -58,8 +60,11 @@ namespace tc {
 constexpr int kWidth = 576;                 // r + d_rope at r = 512
 constexpr int kChunks = 9;                  // 64-column chunks of a row at r = 512 (8 latent + 1 rope)
 constexpr int kGroupPages = 4;              // pages per pair step (256 tokens)
-// warps: 0 Q/QK loads, 1 QK MMA, 2 V loads, 3-6 softmax, 7 PV MMA
+// warps: 0 Q/QK loads, 1 QK MMA, 2 V loads, 3-6 softmax, 7 PV MMA; two
+// latent shards add warps 8-11, the softmax of shard 1 (warps 3-6: shard 0)
 constexpr int kThreads = 256;
+template <int S>
+constexpr int threads_of() { return S == 2 ? 384 : 256; }
 constexpr uint32_t kQChunkBytes = 64 * 128;  // 64 rows x 128 B
 constexpr uint32_t kQBytes = kChunks * kQChunkBytes;
 // The latent width R of one launch: 512 (every workload on one GPU), or 256
@@ -279,7 +284,7 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk16) {
 }
 
 template <int S, int R, bool kSkip = false>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<S>(), 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_q, RunParams p) {
   using namespace ptx;
@@ -330,7 +335,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     counts[B_S_FREE] = counts[B_S_FREE + 1] = 8;
     counts[B_P_FULL] = counts[B_P_FULL_1] = 8;
     counts[B_P_FULL_HI] = counts[B_P_FULL_HI_1] = 4;
-    counts[B_O_FREE] = 8;
+    counts[B_O_FREE] = 8 * S;  // every softmax warp of both CTAs
     counts[B_VSEEN] = counts[B_VSEEN + 1] = 2;  // both CTAs' V producers
     for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), counts[i]);
     fence_mbarrier_init_cluster();
@@ -620,6 +625,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // Every softmax thread executes the same sequence of named barriers
     // whatever happens: after a failed (timed-out) wait the flag `ok` turns
     // false for the whole warp and the remaining groups only skip their work.
+    // two shards: one softmax warpgroup per shard (warps 3-6 and 8-11), each
+    // with its own named barrier; one shard: warps 3-6
+    const int my_shard = (S == 2 && warp >= 8) ? 1 : 0;
     const int lq = (warp & 3) * 32 + lane;         // tensor-memory lane of this thread
     const int half = lq >> 6;                      // token half: group tokens [128 half, +128)
     const int rloc = lq & 63;                      // row within this CTA's 64
@@ -629,7 +637,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     bool ok = true;
     float* xl = xch + 2 * S * 128;                 // [S][128]
-    auto named_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
+    const uint32_t sync_id = 1u + 2u * (uint32_t)my_shard;
+    auto named_sync = [sync_id] { asm volatile("bar.sync %0, 128;" :: "r"(sync_id) : "memory"); };
     auto wait = [&](int b, uint32_t parity) {
       if (ok && *abort_flag) ok = false;
       if (ok) ok = mbar_wait(bar(b), parity, p.wait_limit_ns);
@@ -638,12 +647,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     GroupCursor g;
     bool have = g.init(p, w);
     int gi = 0;
-    float m[S], l[S];
+    float m_run = -INFINITY, l_run = 0.f;  // this thread's row: running max (log2 units) and sum
     float mm = -INFINITY;  // threshold skipping: the row's true running max of the segment (log2 units)
     while (have) {
       if (g.first) {
-#pragma unroll
-        for (int s = 0; s < S; ++s) { m[s] = -INFINITY; l[s] = 0.f; }
+        m_run = -INFINITY;
+        l_run = 0.f;
         mm = -INFINITY;
       }
       const int sb = gi % C::kSBufs;
@@ -666,42 +675,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (ok) tc_fence_after();
       }
 #pragma unroll 1
-      for (int s = 0; s < S; ++s) {
+      for (int s = my_shard; s <= my_shard; ++s) {  // this warpgroup's shard
         if constexpr (S == 2) {
           // two shards: each tile is complete (and released) on its own
           wait(B_S_FULL + s, gi & 1);
           if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_S_READY, gi);
           if (ok) tc_fence_after();
         }
-        // one pass over tensor memory: the thread's 128 scores of shard s
-        uint32_t r[128];
-        if (ok) {
+        // The thread's 128 scores of shard s. One shard: one pass over tensor
+        // memory into registers. Two shards (a warpgroup each, 384 threads,
+        // 168 registers): two passes in 32-column pieces, for the row max and
+        // then for P, so that no 128-score array is live; the tile is released
+        // after the second.
+        const uint32_t s_addr = tbase + lane_off + sb * 128 * S + 128 * s;
+        constexpr int kRegScores = S == 2 ? 1 : 128;
+        uint32_t r[kRegScores];
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+        if constexpr (S == 2) {
+          if (ok) {
 #pragma unroll
-          for (int c0 = 0; c0 < 128; c0 += 32)
-            tmem_ld32(tbase + lane_off + sb * 128 * S + 128 * s + c0,
-                      *reinterpret_cast<uint32_t(*)[32]>(r + c0));
-          tmem_wait_ld();
-        }
-        if (S == 2 || s == S - 1) {
-          // every score of this S buffer (two shards: of this shard's tile)
-          // is in registers: QK may reuse it
+            for (int c0 = 0; c0 < 128; c0 += 64) {
+              uint32_t v[64];
+              tmem_ld32(s_addr + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
+              tmem_ld32(s_addr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+              tmem_wait_ld();
+              // masked keys (past the group or the causal limit) count as -inf
+              if (nvis >= 128) {
+#pragma unroll
+                for (int k = 0; k < 64; k += 2) {
+                  mx0 = fmaxf(mx0, __uint_as_float(v[k]));
+                  mx1 = fmaxf(mx1, __uint_as_float(v[k + 1]));
+                }
+              } else {
+#pragma unroll
+                for (int k = 0; k < 64; k += 2) {
+                  mx0 = fmaxf(mx0, c0 + k < nvis ? __uint_as_float(v[k]) : -INFINITY);
+                  mx1 = fmaxf(mx1, c0 + k + 1 < nvis ? __uint_as_float(v[k + 1]) : -INFINITY);
+                }
+              }
+            }
+          }
+        } else {
+          if (ok) {
+#pragma unroll
+            for (int c0 = 0; c0 < 128; c0 += 32)
+              tmem_ld32(s_addr + c0, *reinterpret_cast<uint32_t(*)[32]>(r + c0));
+            tmem_wait_ld();
+          }
+          // every score of this S buffer is in registers: QK may reuse it
           if (ok) tc_fence_before();
           __syncwarp();
-          if (ok && lane == 0 && !p.withhold_s_free) arrive_leader(B_S_FREE + (S == 2 ? s : sb));
-        }
-        // masked keys (past the group or the causal limit) become -inf: they
-        // drop out of the max and 2^-inf = 0 in the sum and in P
-        if (nvis < 128) {
+          if (ok && lane == 0 && !p.withhold_s_free) arrive_leader(B_S_FREE + sb);
+          // masked keys (past the group or the causal limit) become -inf: they
+          // drop out of the max and 2^-inf = 0 in the sum and in P
+          if (nvis < 128) {
 #pragma unroll
-          for (int j = 0; j < 128; ++j)
-            if (j >= nvis) r[j] = 0xff800000u;
-        }
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-        if (ok) {
+            for (int j = 0; j < 128; ++j)
+              if (j >= nvis) r[j] = 0xff800000u;
+          }
+          if (ok) {
 #pragma unroll
-          for (int j = 0; j < 128; j += 2) {
-            mx0 = fmaxf(mx0, __uint_as_float(r[j]));
-            mx1 = fmaxf(mx1, __uint_as_float(r[j + 1]));
+            for (int j = 0; j < 128; j += 2) {
+              mx0 = fmaxf(mx0, __uint_as_float(r[j]));
+              mx1 = fmaxf(mx1, __uint_as_float(r[j + 1]));
+            }
           }
         }
         const float mt_own = fmaxf(mx0, mx1) * p.scale_log2;
@@ -739,33 +776,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           wait(B_DECIDE + par, (gi >> 1) & 1);
           skip = ok && !pair_keeps(gi);
         }
-        float mu = m[s];
-        if (!skip && (m[s] == -INFINITY || mt > m[s] + kRescaleThreshold)) mu = fmaxf(mt, m[s]);
+        float mu = m_run;
+        if (!skip && (m_run == -INFINITY || mt > m_run + kRescaleThreshold)) mu = fmaxf(mt, m_run);
         float alpha = 1.f;
-        const bool rescale = mu != m[s] && m[s] != -INFINITY;
-        if (rescale) alpha = ex2_approx(m[s] - mu);
-        m[s] = mu;
+        const bool rescale = mu != m_run && m_run != -INFINITY;
+        if (rescale) alpha = ex2_approx(m_run - mu);
+        m_run = mu;
         // P = 2^(score * scale - m) in bf16 pairs, row sum in four partial sums
         // (a row that has seen no key yet keeps m = -inf, all its scores are
         // -inf and P = 0)
         uint32_t pk[64];
         float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
         const float nmu = mu == -INFINITY ? 0.f : -mu;
-        if (!skip) {
-#pragma unroll
-        for (int j = 0; j < 128; j += 4) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, nmu));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, nmu));
-          const float p2 = ex2_approx(fmaf(__uint_as_float(r[j + 2]), p.scale_log2, nmu));
-          const float p3 = ex2_approx(fmaf(__uint_as_float(r[j + 3]), p.scale_log2, nmu));
+        auto p_of4 = [&](int j, float x0, float x1, float x2, float x3) {
+          const float p0 = ex2_approx(fmaf(x0, p.scale_log2, nmu));
+          const float p1 = ex2_approx(fmaf(x1, p.scale_log2, nmu));
+          const float p2 = ex2_approx(fmaf(x2, p.scale_log2, nmu));
+          const float p3 = ex2_approx(fmaf(x3, p.scale_log2, nmu));
           ps0 += p0; ps1 += p1; ps2 += p2; ps3 += p3;
           __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
           __nv_bfloat162 h1 = __floats2bfloat162_rn(p2, p3);
           pk[j >> 1] = *reinterpret_cast<uint32_t*>(&h0);
           pk[(j >> 1) + 1] = *reinterpret_cast<uint32_t*>(&h1);
+        };
+        if constexpr (S == 2) {
+          // second pass over the tile, 32 columns at a time; then release it
+          if (ok) {
+#pragma unroll
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+              uint32_t v[32];
+              tmem_ld32(s_addr + c0, v);
+              tmem_wait_ld();
+              if (nvis >= 128) {
+#pragma unroll
+                for (int k = 0; k < 32; k += 4)
+                  p_of4(c0 + k, __uint_as_float(v[k]), __uint_as_float(v[k + 1]), __uint_as_float(v[k + 2]),
+                        __uint_as_float(v[k + 3]));
+              } else {
+#pragma unroll
+                for (int k = 0; k < 32; k += 4) {
+                  const int j = c0 + k;
+                  p_of4(j, j < nvis ? __uint_as_float(v[k]) : -INFINITY,
+                        j + 1 < nvis ? __uint_as_float(v[k + 1]) : -INFINITY,
+                        j + 2 < nvis ? __uint_as_float(v[k + 2]) : -INFINITY,
+                        j + 3 < nvis ? __uint_as_float(v[k + 3]) : -INFINITY);
+                }
+              }
+            }
+            tc_fence_before();
+          }
+          __syncwarp();
+          if (ok && lane == 0 && !p.withhold_s_free) arrive_leader(B_S_FREE + s);
+        } else if (!skip) {
+#pragma unroll
+          for (int j = 0; j < 128; j += 4)
+            p_of4(j, __uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                  __uint_as_float(r[j + 3]));
         }
-        }
-        l[s] = l[s] * alpha + ((ps0 + ps1) + (ps2 + ps3));
+        l_run = l_run * alpha + ((ps0 + ps1) + (ps2 + ps3));
         if (lq == 0 && s == 0) MLA_TRACE_EV(w, rank, EV_PASS2, gi);
         auto rescale_o = [&](int c0, int ncols) {
           tc_fence_after();
@@ -826,18 +894,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         wait(B_PV_DONE, gi & 1);
         if (lq == 0) MLA_TRACE_EV(w, rank, EV_SYNC1, gi);
         if (ok) tc_fence_after();
-#pragma unroll
-        for (int s = 0; s < S; ++s) xl[s * 128 + lq] = l[s];
+        // (this warpgroup's shard: its l, log2-sum-exp and O columns)
+        const int s = my_shard;
+        xl[s * 128 + lq] = l_run;
         named_sync();
-        float inv[S];
         const int64_t slot = w + g.b;
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
-          const float lt = l[s] + xl[s * 128 + (lq ^ 64)];
-          inv[s] = lt > 0.f ? 1.f / lt : 0.f;
-          if (ok && half == 0 && row_real)
-            p.lse_part[(slot * p.rows + row) * S + s] = lt > 0.f ? m[s] + log2f(lt) : kEmptyLse;
-        }
+        const float lt = l_run + xl[s * 128 + (lq ^ 64)];
+        const float iv = lt > 0.f ? 1.f / lt : 0.f;
+        if (ok && half == 0 && row_real)
+          p.lse_part[(slot * p.rows + row) * S + s] = lt > 0.f ? m_run + log2f(lt) : kEmptyLse;
         if (ok) {
           // O / l goes out as fp16 (the combine kernel reads it back once).
           // A warp holds 32 consecutive rows; per round it loads 64 columns of
@@ -845,18 +910,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // through 4 KB of the P buffer (free: this group's PV has completed),
           // so that each store instruction writes four whole 128-byte row
           // segments. Swizzle: 16-byte unit u of staged row r sits at u ^ (r & 7).
-          uint8_t* stage = gbase + L::p + (warp & 3) * 4096;
+          uint8_t* stage = gbase + L::p + s * C::kPShard + (warp & 3) * 4096;
           const int rbase = 64 * (int)rank + 32 * ((warp & 3) & 1);  // row of lane 0
           const int j = lane & 7;
           __half* oh = reinterpret_cast<__half*>(p.o_part);
+          constexpr int kCols = (int)Wd::kOCols / S;  // this shard's O columns
 #pragma unroll 1
-          for (int c = 0; c < (int)Wd::kOCols; c += 64) {
+          for (int c = kCols * s; c < kCols * (s + 1); c += 64) {
             uint32_t o[64];
             tmem_ld32(tbase + lane_off + kTmemO + c, *reinterpret_cast<uint32_t(*)[32]>(o));
             tmem_ld32(tbase + lane_off + kTmemO + c + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
             tmem_wait_ld();
             const int nb = c >> 7;
-            const float iv = inv[S == 2 ? nb : 0];
             const int col0 = 256 * nb + 128 * half + (c & 127);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -884,6 +949,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           __threadfence();  // this thread's partial rows, before the CTA's segment-done count
         }
         named_sync();  // xl and the O reads of all four warps are done
+        // one count per CTA and shard: the combine waits for 2 S per segment
         if (ok && lq == 0) publish_segment_half(p.seg_done + g.b);
         if (lq == 0) MLA_TRACE_EV(w, rank, EV_LD0, gi);
         __syncwarp();
@@ -945,7 +1011,7 @@ inline cudaError_t launch_decode_variant(const RunParams& p, const CUtensorMap& 
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_tc_kernel<S, R, kSkip>),
                                     (int)Smem<S, R>::alloc);
   if (e != cudaSuccess) return e;
-  return launch_dependent_opt(pdl, decode_tc_kernel<S, R, kSkip>, dim3(2 * p.W), dim3(kThreads), Smem<S, R>::alloc,
+  return launch_dependent_opt(pdl, decode_tc_kernel<S, R, kSkip>, dim3(2 * p.W), dim3(threads_of<S>()), Smem<S, R>::alloc,
                               stream, tm_kv, tm_q, p);
 }
 }  // namespace tc

@@ -289,8 +289,9 @@ __global__ void __launch_bounds__(kCombineThreads, 1)
         const int sh = c0 / (p.r / S);
         const int64_t lo = page_owner(p.cum[b], b, Gv, p.W) + b;
         const int64_t hi = page_owner(p.cum[b + 1] - 1, b, Gv, p.W) + b;
-        // both CTAs of each of the sequence's segments publish their rows (bounded wait)
-        const int32_t want = 2 * (int32_t)(hi - lo + 1);
+        // both CTAs of each of the sequence's segments publish their rows, once
+        // per latent shard (bounded wait)
+        const int32_t want = 2 * S * (int32_t)(hi - lo + 1);
         if (load_acquire_gpu(p.seg_done + b) < want) {
           const uint64_t t0 = ptx::globaltimer_ns();
           bool waited = true;
