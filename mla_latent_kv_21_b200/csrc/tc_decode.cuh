@@ -14,7 +14,7 @@
 //       N = 256 matters: a tcgen05.mma costs ~60 cycles whatever its size, and
 //       only N = 256 (64 rows x 256 x 16 per SM = 64 cycles of math) keeps the
 //       tensor pipe efficient.
-//   softmax (4 warps per CTA, fp32, log2 domain): per row online max / sum;
+//   softmax (4 warps per CTA and shard, fp32, log2 domain): per row online max / sum;
 //       the max is moved (and O rescaled) only when it grows by more than 2^8,
 //       so every P value lies in [0, 256] and rescales are rare. One pass
 //       over the thread's 128 scores in tensor memory (exp2 on the SFU), the
@@ -148,7 +148,7 @@ enum : int {
   B_V_FULL = 7,       // [6] leader, count 2 (+tx)
   B_S_FREE = 13,      // [2] leader, count 8 (4 softmax warps x 2 CTAs): by S buffer (one shard) or by shard
   B_P_FULL = 15,      // leader, count 8: P pages 0, 1 written (2 warps x 2 CTAs) and O rescaled (all 8)
-  B_O_FREE = 16,      // leader, count 8
+  B_O_FREE = 16,      // leader, count 8 S (every softmax warp of both CTAs)
   B_QK_FREE = 17,     // [6] both, count 1 (MMA commit)
   B_V_FREE = 23,      // [6] both, count 1
   B_S_FULL = 29,      // [2] both, count 1: by S buffer (one shard) or by shard (two)
@@ -948,7 +948,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<S>(), 1)
           tc_fence_before();
           __threadfence();  // this thread's partial rows, before the CTA's segment-done count
         }
-        named_sync();  // xl and the O reads of all four warps are done
+        named_sync();  // xl and the O reads of the warpgroup's four warps are done
         // one count per CTA and shard: the combine waits for 2 S per segment
         if (ok && lq == 0) publish_segment_half(p.seg_done + g.b);
         if (lq == 0) MLA_TRACE_EV(w, rank, EV_LD0, gi);
