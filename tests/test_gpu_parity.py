@@ -49,6 +49,38 @@ def test_reduced_size_parity(cuda_device, name, lens, kernel):
     assert_close(got.double().numpy(), ref, wl.dtype, f"{name} {lens} kernel={info.kernel}")
 
 
+@pytest.mark.parametrize("heads,q_len,lens", [
+    (64, 2, [2, 3, 65, 66, 130, 700]),   # two query tokens: causal limit per query row
+    (16, 1, [1, 64, 65, 257, 900]),      # 16 real rows of each CTA pair's 128
+    (128, 1, [4096, 33]),                # several segments per sequence
+])
+def test_two_shard_shapes(cuda_device, heads, q_len, lens):
+    """The two-shard (TPLA) decode on shapes beyond its workload: MTP rows,
+    few heads, long sequences split over several workers; every element."""
+    wl = WORKLOADS["tpla_dsv3"].with_(heads=heads, q_len=q_len)
+    inputs = generate(wl, seq_lens=lens)
+    got, info = run_gpu(wl, inputs, cuda_device)
+    assert info.kernel == M.MLA_KERNEL_TCGEN05
+    ref = oracle_out(wl, inputs)
+    assert_close(got.double().numpy(), ref, wl.dtype, f"two shards H={heads} Lq={q_len} {lens}")
+
+
+@pytest.mark.parametrize("heads,q_len,lens", [
+    (40, 1, [1, 65, 300, 2000]),     # 40 rows: the second CTA of each pair holds only padding rows
+    (96, 1, [3, 64, 129, 1500]),     # 96 rows: the second CTA holds 32 real rows
+    (48, 2, [2, 5, 190, 777]),       # 96 rows over two query tokens
+])
+def test_one_shard_row_counts(cuda_device, heads, q_len, lens):
+    """The one-shard decode at row counts (heads x query tokens) between the
+    workloads' 32, 128: every element."""
+    wl = WORKLOADS["deepseek_v3"].with_(heads=heads, q_len=q_len)
+    inputs = generate(wl, seq_lens=lens)
+    got, info = run_gpu(wl, inputs, cuda_device)
+    assert info.kernel == M.MLA_KERNEL_TCGEN05
+    ref = oracle_out(wl, inputs)
+    assert_close(got.double().numpy(), ref, wl.dtype, f"one shard H={heads} Lq={q_len} {lens}")
+
+
 def full_size_pairs(wl, n_min=64):
     """(sequence, head) pairs checked at full size: every sequence (so every
     split segment, including those of workers whose range crosses a sequence
