@@ -139,6 +139,7 @@ struct Smem {
   static_assert(Cfg<S, R>::kQkSlots <= 6 && Cfg<S, R>::kVSlots <= 6, "barrier arrays hold 6 slots");
   static constexpr uint32_t total = misc + 64;
   static constexpr uint32_t alloc = total + 1024;     // alignment slack
+  static_assert(alloc <= 227 * 1024, "shared memory of one CTA");
 };
 
 // barrier indices (leader = only the leader CTA's copy is used)

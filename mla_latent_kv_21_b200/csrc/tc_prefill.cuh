@@ -74,6 +74,7 @@ struct UpSmem {
   static constexpr uint32_t bars = ring + kStages * kStageBytes;
   static constexpr uint32_t misc = bars + 128;
   static constexpr uint32_t alloc = misc + 64 + 1024;
+  static_assert(alloc <= 227 * 1024, "shared memory of one CTA");
 };
 enum : int { U_A_FULL = 0, U_B_FULL = 1, U_B_EMPTY = 4, U_D_FULL = 7, U_D_EMPTY = 9, U_COUNT = 11 };
 
@@ -243,6 +244,7 @@ struct AttnSmem {
   static constexpr uint32_t bars = pbuf + 2 * 16384;
   static constexpr uint32_t misc = bars + 256;
   static constexpr uint32_t alloc = misc + 64 + 1024;
+  static_assert(alloc <= 227 * 1024, "shared memory of one CTA");
 };
 enum : int {
   A_Q_FULL = 0, A_K_FULL = 1, A_K_EMPTY = 6, A_V_FULL = 11, A_V_EMPTY = 13, A_S_FULL = 15,
