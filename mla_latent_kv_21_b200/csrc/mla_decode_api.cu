@@ -515,6 +515,11 @@ int mla_debug_trace_hg_read(unsigned long long* host, size_t n) {
   if (n > cap) n = cap;
   return cudaMemcpyFromSymbol(host, hg::g_hg_trace, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 1;
 }
+int mla_debug_trace_pf_read(unsigned long long* host, size_t n) {
+  const size_t cap = sizeof(pf::g_pf_trace) / sizeof(unsigned long long);
+  if (n > cap) n = cap;
+  return cudaMemcpyFromSymbol(host, pf::g_pf_trace, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : 1;
+}
 int mla_debug_trace_chunks_read(unsigned long long* host, size_t n) {
   const size_t cap = sizeof(tc::g_trace_chunk) / sizeof(unsigned long long);
   if (n > cap) n = cap;

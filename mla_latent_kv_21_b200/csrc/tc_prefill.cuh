@@ -252,6 +252,27 @@ enum : int {
 };
 constexpr float kPrefillRescaleThreshold = 8.0f;  // log2 units
 
+// Optional event trace (compile with -DMLA_TRACE): SM clock of per-item
+// events of the first attention CTA (its longest query tile), read back with
+// mla_debug_trace_pf_read(). Kinds: 0 K item load issued, 1 K item seen full
+// by the MMA issuer, 2 V tile load issued, 3 P seen full by the MMA issuer,
+// 4 V seen full (PV issued), 5 S seen full by the softmax, 6 the softmax may
+// write P, 7 P written.
+#ifdef MLA_TRACE
+constexpr int kPfTraceItems = 256;
+__device__ unsigned long long g_pf_trace[8 * kPfTraceItems];
+#define MLA_PF_TRACE(kind, idx)                                                          \
+  do {                                                                                   \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (idx) < kPfTraceItems) { \
+      unsigned long long t_;                                                             \
+      asm volatile("mov.u64 %0, %%clock64;" : "=l"(t_));                                 \
+      g_pf_trace[(kind) * kPfTraceItems + (idx)] = t_;                                   \
+    }                                                                                    \
+  } while (0)
+#else
+#define MLA_PF_TRACE(kind, idx) do {} while (0)
+#endif
+
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_qr,
                 const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_kr,
@@ -316,6 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = mbar_wait(bar(A_K_EMPTY + slot), ((kc / AttnSmem::kKSlots) - 1) & 1, p.wait_limit_ns);
           if (!ok) break;
           const uint32_t dst = base + AttnSmem::k + slot * 16384;
+          MLA_PF_TRACE(0, kc);
           mbar_arrive_expect_tx_local(bar(A_K_FULL + slot), 16384);
           if (i < 2) tma_load_2d(dst, &tm_kn, 64 * i, krow, bar(A_K_FULL + slot));
           else tma_load_2d(dst, &tm_kr, p.r, key0, bar(A_K_FULL + slot));  // k_rope: latent-row columns [r, r + 64)
@@ -326,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(bar(A_V_EMPTY + vs), ((j / AttnSmem::kVSlots) - 1) & 1, p.wait_limit_ns);
         if (!ok) break;
         const uint32_t dst = base + AttnSmem::v + vs * 32768;
+        MLA_PF_TRACE(2, j);
         mbar_arrive_expect_tx_local(bar(A_V_FULL + vs), 32768);
         tma_load_2d(dst, &tm_v, 0, krow, bar(A_V_FULL + vs));
         tma_load_2d(dst + 16384, &tm_v, 64, krow, bar(A_V_FULL + vs));
@@ -351,6 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int slot = kc % AttnSmem::kKSlots;
           ok = mbar_wait(bar(A_K_FULL + slot), (kc / AttnSmem::kKSlots) & 1, p.wait_limit_ns);
           if (!ok) break;
+          MLA_PF_TRACE(1, kc);
           tc_fence_after();
           const uint64_t ad = q_desc + (uint64_t)((i * 16384) >> 4);
           const uint64_t bd = k_desc + (uint64_t)((slot * 16384) >> 4);
@@ -367,9 +391,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j + 1 < nkt) issue_qk(j + 1);
         if (!ok) break;
         const int vs = j % AttnSmem::kVSlots;
-        ok = mbar_wait(bar(A_P_FULL), j & 1, p.wait_limit_ns) &&
-             mbar_wait(bar(A_V_FULL + vs), (j / AttnSmem::kVSlots) & 1, p.wait_limit_ns);
+        ok = mbar_wait(bar(A_P_FULL), j & 1, p.wait_limit_ns);
+        MLA_PF_TRACE(3, j);
+        ok = ok && mbar_wait(bar(A_V_FULL + vs), (j / AttnSmem::kVSlots) & 1, p.wait_limit_ns);
         if (!ok) break;
+        MLA_PF_TRACE(4, j);
         tc_fence_after();
         const uint64_t vd = v_desc + (uint64_t)((vs * 32768) >> 4);
 #pragma unroll
@@ -397,6 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < nkt; ++j) {
       const int sb = j & 1;
       wait(A_S_FULL + sb, (j >> 1) & 1);
+      if (row == 0) MLA_PF_TRACE(5, j);
       uint32_t r[128];
       if (ok) {
         tc_fence_after();
@@ -449,6 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
       // the PV of tile j - 1 is done with P and has added to O
       if (j >= 1) wait(A_P_EMPTY, (j - 1) & 1);
+      if (row == 0) MLA_PF_TRACE(6, j);
       if (ok && j >= 1 && __any_sync(0xffffffffu, rescale)) {
         tc_fence_after();
 #pragma unroll 1
@@ -477,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (ok && lane == 0) mbar_arrive_local(bar(A_P_FULL));
+      if (row == 0) MLA_PF_TRACE(7, j);
     }
     // ---- epilogue: O / l of this row
     wait(A_P_EMPTY, (nkt - 1) & 1);
