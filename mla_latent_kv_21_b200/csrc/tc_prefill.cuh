@@ -26,8 +26,8 @@
 //          V tiles (32 KB, MN-major). S = Q K^T (M = 128, N = 128, K = 192) in
 //          one of two tensor-memory buffers; four softmax warps (one query
 //          row per thread, fp32, log2 domain, lazy max with threshold 2^8)
-//          write P (bf16) to shared memory; O += P V (N = 128, K = 128) in
-//          tensor memory. The QK of tile j + 1 is issued before the PV of
+//          write P (bf16 pairs) to tensor memory; O += P V (N = 128, K = 128)
+//          in tensor memory, P the MMA's A operand straight from there. The QK of tile j + 1 is issued before the PV of
 //          tile j, so the tensor core works while the softmax of tile j runs.
 //
 // Every wait is bounded (p.wait_limit_ns) and records MLA_ERR_DEVICE_TIMEOUT.
@@ -240,8 +240,7 @@ struct AttnSmem {
   static constexpr int kVSlots = 2;                   // 32 KB: V tile, two 64-column halves
   static constexpr uint32_t k = 3 * 16384;
   static constexpr uint32_t v = k + kKSlots * 16384;
-  static constexpr uint32_t pbuf = v + kVSlots * 32768;  // 2 chunks x [128 rows][64 keys] bf16
-  static constexpr uint32_t bars = pbuf + 2 * 16384;
+  static constexpr uint32_t bars = v + kVSlots * 32768;
   static constexpr uint32_t misc = bars + 256;
   static constexpr uint32_t alloc = misc + 64 + 1024;
   static_assert(alloc <= 227 * 1024, "shared memory of one CTA");
@@ -251,6 +250,18 @@ enum : int {
   A_S_EMPTY = 17, A_P_FULL = 19, A_P_EMPTY = 20, A_COUNT = 21
 };
 constexpr float kPrefillRescaleThreshold = 8.0f;  // log2 units
+
+// D += A x B with A in tensor memory (cta_group::1): A's M rows are the lanes
+// from a_tmem on, its K elements run along the columns, two 16-bit elements
+// per 32-bit column (element 2c in the low half of column c); B is a shared
+// memory descriptor as for ptx::mma_f16.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      :: "r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
 
 // Optional event trace (compile with -DMLA_TRACE): SM clock of per-item
 // events of the first attention CTA (its longest query tile), read back with
@@ -309,7 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  const uint32_t kTmemO = 256;
+  const uint32_t kTmemO = 256;  // O: columns [256, 384); S: two buffers of 128 columns from 0
+  const uint32_t kTmemP = 384;  // P (bf16 pairs): columns [384, 448), the A operand of P V
   bool ok = true;
 
   if (warp == 0) {
@@ -364,7 +376,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t q_desc = smem_desc_sw128(base + AttnSmem::q, 16, 1024);
       const uint64_t k_desc = smem_desc_sw128(base + AttnSmem::k, 16, 1024);
       const uint64_t v_desc = smem_desc_sw128(base + AttnSmem::v, 16384, 1024);
-      const uint64_t p_desc = smem_desc_sw128(base + AttnSmem::pbuf, 16, 1024);
       uint32_t kc = 0;
       ok = mbar_wait(bar(A_Q_FULL), 0, p.wait_limit_ns);
       auto issue_qk = [&](int j) {
@@ -399,9 +410,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint64_t vd = v_desc + (uint64_t)((vs * 32768) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_f16<1>(tbase + kTmemO, p_desc + (uint64_t)(((ks >> 2) * 16384) >> 4) + (uint64_t)(2 * (ks & 3)),
-                     vd + (uint64_t)(128 * ks), idesc_o, (j | ks) ? 1u : 0u);
+        for (int ks = 0; ks < 8; ++ks)  // K = 16 keys per MMA: 8 columns of P
+          mma_f16_ts(tbase + kTmemO, tbase + kTmemP + 8 * ks, vd + (uint64_t)(128 * ks), idesc_o,
+                     (j | ks) ? 1u : 0u);
         tc_commit<1>(bar(A_V_EMPTY + vs));
         tc_commit<1>(bar(A_P_EMPTY));
       }
@@ -491,16 +502,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       if (ok) {
-        // P row -> shared memory, K-major 128-byte swizzle: keys [64 t, +64) in chunk t
-        uint8_t* pb = gbase + AttnSmem::pbuf;
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(pb + t * 16384 + sw128(row, u)) =
-                make_uint4(pk[32 * t + 4 * u], pk[32 * t + 4 * u + 1], pk[32 * t + 4 * u + 2],
-                           pk[32 * t + 4 * u + 3]);
-        fence_proxy_async_smem();
+        // P row -> tensor memory: this thread's lane, keys 2c and 2c + 1 in column c
+        tmem_st32(tbase + lane_off + kTmemP, *reinterpret_cast<uint32_t(*)[32]>(pk));
+        tmem_st32(tbase + lane_off + kTmemP + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+        tmem_wait_st();
         tc_fence_before();
       }
       __syncwarp();
