@@ -7,7 +7,9 @@
   with 8 workers that each cross several sequence ends (segments of one or
   two pages, partial groups, query reloads);
 * two plans of different workloads run concurrently on two streams with their
-  own workspaces: results equal the same runs made one after the other.
+  own workspaces: results equal the same runs made one after the other;
+* seeded random shapes (heads, query tokens, latent shards, worker count and
+  lengths drawn together) on the tensor-core path, every element.
 """
 
 import random
@@ -91,3 +93,31 @@ def test_tail_slots_may_hold_any_rope_and_finite_ckv(cuda_device):
     assert torch.isfinite(dirty.float()).all()
     assert torch.equal(clean, dirty)
 
+
+
+def _random_shapes(n=8, seed=2024):
+    rng = random.Random(seed)
+    cases = []
+    for _ in range(n):
+        shards = rng.choice([1, 2])
+        q_len = rng.choice([1, 1, 2])
+        heads = rng.choice([h for h in (8, 16, 24, 40, 64, 96, 128) if h * q_len <= 128])
+        lens = [rng.randint(q_len, rng.choice([70, 700, 3000])) for _ in range(rng.randint(1, 6))]
+        workers = rng.choice([0, 0, 5, 33])
+        cases.append((shards, q_len, heads, lens, workers))
+    return cases
+
+
+@pytest.mark.parametrize("shards,q_len,heads,lens,workers", _random_shapes())
+def test_random_shapes(cuda_device, shards, q_len, heads, lens, workers):
+    """Heads x query tokens from 8 to 128 rows, one or two latent shards,
+    default and small worker counts, ragged lengths: the tensor-core path
+    against the oracle, every element."""
+    base = WORKLOADS["tpla_dsv3" if shards == 2 else "deepseek_v3"]
+    wl = base.with_(heads=heads, q_len=q_len)
+    inputs = generate(wl, seq_lens=lens)
+    got, info = run_gpu(wl, inputs, cuda_device, num_workers=workers)
+    assert info.kernel == M.MLA_KERNEL_TCGEN05
+    ref = oracle_out(wl, inputs)
+    assert_close(got.double().numpy(), ref, wl.dtype,
+                 f"S={shards} H={heads} Lq={q_len} workers={info.num_workers} {lens}")
