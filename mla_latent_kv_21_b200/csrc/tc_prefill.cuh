@@ -251,6 +251,33 @@ enum : int {
 };
 constexpr float kPrefillRescaleThreshold = 8.0f;  // log2 units
 
+// Paired float arithmetic of sm_100 (one instruction for two lanes' worth of
+// work, each element rounded as the scalar instruction rounds it) and the
+// three-input max: the softmax issues fewer instructions per score.
+__device__ __forceinline__ uint64_t pair_f32(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpair_f32(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // D += A x B with A in tensor memory (cta_group::1): A's M rows are the lanes
 // from a_tmem on, its K elements run along the columns, two 16-bit elements
 // per 32-bit column (element 2c in the low half of column c); B is a shared
@@ -458,9 +485,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        mx0 = fmaxf(mx0, __uint_as_float(r[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(r[c + 1]));
+      for (int c = 0; c < 128; c += 4) {
+        mx0 = max3(mx0, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+        mx1 = max3(mx1, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
       }
       const float mt = fmaxf(mx0, mx1) * p.scale_log2;
       float mu = m;
@@ -471,19 +498,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       m = mu;
       const float nmu = mu == -INFINITY ? 0.f : -mu;
       uint32_t pk[64];
-      float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
+      // two pairs of running sums (the same four sums, added pairwise)
+      uint64_t ps01 = pair_f32(0.f, 0.f), ps23 = pair_f32(0.f, 0.f);
+      const uint64_t sc2 = pair_f32(p.scale_log2, p.scale_log2), nmu2 = pair_f32(nmu, nmu);
 #pragma unroll
       for (int c = 0; c < 128; c += 4) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(r[c]), p.scale_log2, nmu));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), p.scale_log2, nmu));
-        const float p2 = ex2_approx(fmaf(__uint_as_float(r[c + 2]), p.scale_log2, nmu));
-        const float p3 = ex2_approx(fmaf(__uint_as_float(r[c + 3]), p.scale_log2, nmu));
-        ps0 += p0; ps1 += p1; ps2 += p2; ps3 += p3;
+        float x0, x1, x2, x3;
+        unpair_f32(fma2(pair_f32(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sc2, nmu2), x0, x1);
+        unpair_f32(fma2(pair_f32(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])), sc2, nmu2), x2, x3);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+        ps01 = add2(ps01, pair_f32(p0, p1));
+        ps23 = add2(ps23, pair_f32(p2, p3));
         __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
         __nv_bfloat162 h1 = __floats2bfloat162_rn(p2, p3);
         pk[c >> 1] = *reinterpret_cast<uint32_t*>(&h0);
         pk[(c >> 1) + 1] = *reinterpret_cast<uint32_t*>(&h1);
       }
+      float ps0, ps1, ps2, ps3;
+      unpair_f32(ps01, ps0, ps1);
+      unpair_f32(ps23, ps2, ps3);
       l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
       // the PV of tile j - 1 is done with P and has added to O
       if (j >= 1) wait(A_P_EMPTY, (j - 1) & 1);
